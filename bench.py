@@ -1,0 +1,527 @@
+#!/usr/bin/env python
+"""Benchmark of the MXFP8 scale-factor rearrange (per-group 128x4 blocked layout).
+
+One step = one pass of the hot path over one batch of synthetic scales: the
+three production shapes of the pytorch/ao pages, each one C-ABI call:
+  * M-groups (131072, 44), G=8  -- the DSV3-16b shape of #3708 (fallback path)
+  * M-groups (131072, 224), G=8 -- data K = 7168 (TMA path)
+  * K-groups (7168, 4096), G=8  -- data K = 131072 tokens (TMA path)
+Metric: GB/s = (bytes of real scales read + exact padded bytes written) / time,
+and the same as a fraction of the measured HBM copy bandwidth.
+
+Timing: the K timed steps are captured in one CUDA graph (as the pages timed
+their kernels) and replayed once between CUDA events; inputs and outputs
+rotate over enough buffer sets that one rotation spans more than 4x the L2,
+so every step reads cold inputs.  Timing events captured inside the graph
+give each kernel's own duration.  Multi-GPU: independent replicas, one
+process per GPU (torchrun), max time over ranks.
+
+--impl reference times the CPU oracle (the plain C statement of the layout)
+on this host on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+WORKLOADS = {
+    "moe_step": ["m_skinny", "m_wide", "k_groups"],
+    "m_skinny": ["m_skinny"],
+    "m_wide": ["m_wide"],
+    "k_groups": ["k_groups"],
+}
+WORKLOAD_DESC = {
+    "moe_step": "M-groups 131072x44 G=8 (fallback) + M-groups 131072x224 G=8 (TMA) + K-groups 7168x4096 G=8 (TMA)",
+    "m_skinny": "M-groups 131072x44 G=8, stride 44 B (fallback)",
+    "m_wide": "M-groups 131072x224 G=8 (TMA)",
+    "k_groups": "K-groups 7168x4096 G=8 (TMA)",
+}
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2**20
+METRIC = "rearrange GB/s (read+padded write) and % of B200 HBM peak, 1 GPU"
+
+
+# ------------------------------------------------------------------ sizes
+def ceil_to(x: int, a: int) -> int:
+    return -(-x // a) * a
+
+
+def clamped_sizes(ends, limit):
+    e = np.minimum(np.maximum.accumulate(np.maximum(np.asarray(ends, np.int64), 0)), limit)
+    return np.diff(np.concatenate([[0], e])), int(e[-1])
+
+
+def algorithmic_bytes(case) -> dict:
+    """Real input bytes read, exact padded bytes written, and the allocation."""
+    M = case.dim == 0
+    sizes, used = clamped_sizes(case.ends, case.rows if M else case.cols)
+    if M:
+        read = used * case.cols
+        written = sum(ceil_to(int(n), 128) for n in sizes) * ceil_to(case.cols, 4)
+        alloc = (case.rows + 128 * case.num_groups) * ceil_to(case.cols, 4)
+    else:
+        read = case.rows * used
+        written = ceil_to(case.rows, 128) * sum(ceil_to(int(n), 4) for n in sizes)
+        alloc = ceil_to(case.rows, 128) * (case.cols + 4 * case.num_groups)
+    return {"read": int(read), "written": int(written), "alloc": int(alloc)}
+
+
+def make_cases(workload: str):
+    from scale_factor_layout_b200 import synth
+
+    return [synth.NAMED[name]() for name in WORKLOADS[workload]]
+
+
+# ------------------------------------------------------------------ environment
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "scale_factor_layout_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch recorded by an ncu capture (profiles/ncu_traffic.txt),
+    or None when absent or taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = kernel_source_sha()
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        kv = dict(tok.split("=", 1) for tok in line.split() if "=" in tok)
+        if kv.get("call") == kernel and kv.get("source_sha") == sha:
+            return int(float(kv["bytes_per_launch"]))
+    return None
+
+
+class ClockSampler:
+    """Samples SM clocks and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.period, self.index = [], period_s, index
+        self._stop = threading.Event()
+        self.window = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+            self.max_mhz = None
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                mhz = n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM)
+                reasons = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.nvml:
+            self.t.join()
+
+    def summary(self):
+        if not self.nvml or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        t0, t1 = self.window if self.window else (self.samples[0][0], self.samples[-1][0])
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if len(inside) < 3:  # a short timed region: take the samples nearest to it
+            mid = 0.5 * (t0 + t1)
+            inside = sorted(self.samples, key=lambda s: abs(s[0] - mid))[:5]
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        reasons = [name for b, name in self.REASONS.items() if bits & b and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(world: int, backend: str):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, dist, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate_value(bytes_per_step: int, steps: int, n_gpus: int, seconds: float) -> float:
+    """Whole-job GB/s: the bytes all replicas moved over the slowest rank's time."""
+    return bytes_per_step * steps * n_gpus / seconds / 1e9
+
+
+# ------------------------------------------------------------------ GPU arm
+class DeviceSet:
+    """One rotation set: device copies of every case's inputs plus outputs."""
+
+    def __init__(self, cases, device):
+        import torch
+
+        import scale_factor_layout_b200 as mxs
+
+        self.items = []
+        for c in cases:
+            s = torch.from_numpy(np.ascontiguousarray(c.scales)).to(device)
+            e = torch.from_numpy(np.ascontiguousarray(c.ends, dtype=np.int32)).to(device)
+            size = mxs.mx_rearranged_size(c.dim, c.rows, c.cols, c.num_groups)
+            o = torch.empty(size, dtype=torch.uint8, device=device)
+            self.items.append((c, s, e, o))
+
+    def bytes(self):
+        return sum(i[1].numel() + i[3].numel() for i in self.items)
+
+
+def launch(item, stream_handle):
+    from scale_factor_layout_b200 import _binding as B
+
+    c, s, e, o = item
+    st = B.mx_rearrange_ex(c.dim, s.data_ptr(), c.rows, c.cols, c.cols, e.data_ptr(), c.num_groups,
+                           o.data_ptr(), B.MX_PATH_AUTO, stream_handle)
+    if st != B.MX_OK:
+        raise RuntimeError(f"{c.name}: {B.status_string(st)}")
+
+
+def run_ours(args, rank, world, local):
+    import torch
+
+    import scale_factor_layout_b200 as mxs
+    from scale_factor_layout_b200 import _build
+
+    _build.build()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = dist_init(world, "nccl")
+    cases = make_cases(args.workload)
+    per_call = [algorithmic_bytes(c) for c in cases]
+    step_bytes = sum(b["read"] + b["written"] for b in per_call)
+    step_bytes_pages = sum(b["read"] + b["alloc"] for b in per_call)
+
+    first = DeviceSet(cases, device)
+    n_sets = max(2, math.ceil(4 * L2_BYTES / first.bytes()))
+    sets = [first] + [DeviceSet(cases, device) for _ in range(n_sets - 1)]
+    stream = torch.cuda.Stream(device)
+    h = stream.cuda_stream
+    ncalls = len(cases)
+    with torch.cuda.stream(stream):
+        for k in range(3):  # first calls set kernel attributes (outside capture) and warm caches
+            for it in sets[k % n_sets].items:
+                launch(it, h)
+    torch.cuda.synchronize()
+
+    def capture(steps, with_events):
+        g = torch.cuda.CUDAGraph()
+        evs = []
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for k in range(steps):
+                    row = []
+                    for it in sets[k % n_sets].items:
+                        if with_events:
+                            ev = torch.cuda.Event(enable_timing=True, external=True)
+                            ev.record(stream)
+                            row.append(ev)
+                        launch(it, h)
+                    if with_events:
+                        ev = torch.cuda.Event(enable_timing=True, external=True)
+                        ev.record(stream)
+                        row.append(ev)
+                    evs.append(row)
+        return g, evs
+
+    warm_g, _ = capture(args.warmup, False)
+    timed_g, evs = capture(args.steps, True)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+
+    sampler = ClockSampler(local)
+    with sampler:
+        with torch.cuda.stream(stream):
+            warm_g.replay()
+        torch.cuda.synchronize()
+        barrier(dist, device)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            timed_g.replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+        t1 = time.perf_counter()
+        barrier(dist, device)
+        sampler.window = (t0, t1)
+    seconds = start.elapsed_time(end) / 1e3
+    seconds_max = max_over_ranks(seconds, dist, device)
+    # per-kernel durations from the events captured around each call
+    durs = [[r[i].elapsed_time(r[i + 1]) / 1e3 for r in evs] for i in range(ncalls)]
+    avg = [statistics.fmean(d) for d in durs]
+    del timed_g, warm_g
+
+    peak, peak_src = load_peaks()
+    value = aggregate_value(step_bytes, args.steps, world, seconds_max)
+    calls = []
+    for c, b, t in zip(cases, per_call, avg):
+        gbs = (b["read"] + b["written"]) / t / 1e9
+        path = mxs.mx_select_path(c.dim, sets[0].items[cases.index(c)][1].data_ptr(), c.rows, c.cols, c.cols)
+        calls.append({"case": c.name, "path": {1: "tma", 2: "word", 3: "byte"}.get(path, "?"),
+                      "us": round(t * 1e6, 3), "gbps": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
+                      "read_bytes": b["read"], "written_bytes": b["written"], "alloc_bytes": b["alloc"],
+                      "gbps_pages_convention": round((b["read"] + b["alloc"]) / t / 1e9, 1)})
+    dom = max(range(ncalls), key=lambda i: avg[i])
+    dc = calls[dom]
+    achieved = dc["read_bytes"] + dc["written_bytes"]
+    roofline = {"bound": "hbm", "kernel": f"rearrange_tma ({dc['case']})" if dc["path"] == "tma"
+                else f"rearrange_fallback ({dc['case']})",
+                "achieved": round(achieved / avg[dom] / 1e9, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / avg[dom] / 1e9 / peak, 4), "peak_source": f"{peak_src} hbm_gbs",
+                "traffic": ncu_traffic(dc["case"]), "algorithmic_bytes": achieved}
+
+    e2e = run_e2e(args, cases, device, world, dist) if not args.no_e2e else None
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(seconds_max / args.steps * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+        "data": "synthetic (seeded uniform E8M0 bytes, seeded group splits)",
+        "config": {"workload": args.workload, "description": WORKLOAD_DESC[args.workload],
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "bytes_per_step": step_bytes, "bytes_per_step_pages_convention": step_bytes_pages,
+                   "l2": f"rotating {n_sets} input/output sets, {n_sets * first.bytes() / 1e6:.0f} MB > 4x L2",
+                   "timing": "one CUDA graph of all timed steps, CUDA events, max over ranks"},
+        "frac_of_peak": round(value / world / peak, 4),
+        "calls": calls,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": args.steps * ncalls,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(cases, args.cpu_seconds)
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result))
+
+
+def run_e2e(args, cases, device, world, dist):
+    """Through the public torch-level API: pinned host inputs copied in, the
+    rearrange, the output copied back, every step."""
+    import torch
+
+    import scale_factor_layout_b200 as mxs
+
+    host_in = [(torch.from_numpy(np.ascontiguousarray(c.scales)).pin_memory(),
+                torch.from_numpy(np.ascontiguousarray(c.ends, dtype=np.int32)).pin_memory()) for c in cases]
+    dev_in = [(torch.empty(s.shape, dtype=torch.uint8, device=device), torch.empty(e.shape, dtype=torch.int32,
+               device=device)) for s, e in host_in]
+    sizes = [mxs.mx_rearranged_size(c.dim, c.rows, c.cols, c.num_groups) for c in cases]
+    dev_out = [torch.empty(n, dtype=torch.uint8, device=device) for n in sizes]
+    host_out = [torch.empty(n, dtype=torch.uint8).pin_memory() for n in sizes]
+    steps = max(3, min(args.steps, args.e2e_steps))
+
+    def step():
+        for c, (hs, he), (ds, de), do, ho in zip(cases, host_in, dev_in, dev_out, host_out):
+            ds.copy_(hs, non_blocking=True)
+            de.copy_(he, non_blocking=True)
+            mxs.rearrange(c.dim, ds, de, out=do)
+            ho.copy_(do, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    seconds = max_over_ranks(start.elapsed_time(end) / 1e3, dist, device)
+    per_call = [algorithmic_bytes(c) for c in cases]
+    step_bytes = sum(b["read"] + b["written"] for b in per_call)
+    h2d = sum(s.numel() + e.numel() * 4 for s, e in host_in)
+    d2h = sum(sizes)
+    return {"value": round(aggregate_value(step_bytes, steps, world, seconds), 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(seconds / steps * 1e3, 4)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(cases, budget_s: float) -> dict:
+    """The CPU oracle as it stands (single-threaded C), on this host, over
+    whole-call repetitions of the workload until about `budget_s` seconds."""
+    import oracle
+
+    oracle.load()
+    per = [algorithmic_bytes(c) for c in cases]
+    step_bytes = sum(b["read"] + b["written"] for b in per)
+    reps, t_total = 0, 0.0
+    while t_total < budget_s and reps < 1000:
+        t0 = time.perf_counter()
+        for c in cases:
+            oracle.rearrange(c.dim, c.scales, c.ends)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    return {"value": round(step_bytes * reps / t_total / 1e9, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{reps} full steps ({'+'.join(c.name for c in cases)}), {t_total:.1f} s, "
+                      f"single thread, gcc -O2, {os.cpu_count()} host cores ({cpu_model()})"}
+
+
+def sample_cases(cases, fraction: float):
+    """Leading row blocks of each case (offsets clamped by the layout's own rule)."""
+    from scale_factor_layout_b200 import synth
+
+    out = []
+    for c in cases:
+        rows = max(128, int(c.rows * fraction) // 128 * 128) if c.rows >= 128 else c.rows
+        out.append(synth.Case(c.name, c.dim, c.scales[:rows], c.ends.copy(), c.seed))
+    return out
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm (rank 0 only; other ranks exit)."""
+    if rank != 0:
+        return
+    import oracle
+
+    oracle.load()
+    cases = make_cases(args.workload)
+    t0 = time.perf_counter()
+    for c in cases:
+        oracle.rearrange(c.dim, c.scales, c.ends)
+    full_step = time.perf_counter() - t0
+    budget = 120.0
+    fraction = min(1.0, budget / max(1e-9, full_step * (args.steps + args.warmup)))
+    sample = cases if fraction >= 1.0 else sample_cases(cases, fraction)
+    per = [algorithmic_bytes(c) for c in sample]
+    step_bytes = sum(b["read"] + b["written"] for b in per)
+    for _ in range(args.warmup):
+        for c in sample:
+            oracle.rearrange(c.dim, c.scales, c.ends)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for c in sample:
+            oracle.rearrange(c.dim, c.scales, c.ends)
+    seconds = time.perf_counter() - t0
+    value = step_bytes * args.steps / seconds / 1e9
+    desc = "full workload" if fraction >= 1.0 else f"leading {fraction:.3f} of each case's rows"
+    res = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(seconds / args.steps * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+           "data": "synthetic (seeded uniform E8M0 bytes, seeded group splits)",
+           "config": {"workload": args.workload, "description": WORKLOAD_DESC[args.workload],
+                      "parallelism": "single host thread"},
+           "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                            "sample": f"{desc}, single thread, gcc -O2, {cpu_model()}"},
+           "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="moe_step")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+    args.steps = max(1, args.steps)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

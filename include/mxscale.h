@@ -1,0 +1,133 @@
+/*
+ * mxscale.h -- C ABI of libmxscale: MXFP8 E8M0 scale factors -> per-group
+ * 128x4 blocked ("swizzled") layout, on NVIDIA B200 (sm_100a).
+ *
+ * The operation (pytorch/ao pull requests on MXFP8 MoE training):
+ *   - "[mxfp8 moe training] compute prefix sum of group sizes inside kernel
+ *     intead of precomputing" (#3285), Context and Changes: the padded start
+ *     of every group is a prefix sum of padded group sizes, computed inside
+ *     the kernel, with no host precompute and no device-to-host copy.
+ *   - "[mxfp8 moe training] fallback cuda kernel for when input doesn't meet 2d
+ *     TMA constraints" (#3708), Context: groups along M; a pipelined TMA kernel
+ *     when the row stride is a multiple of 16 bytes, a simpler kernel for any
+ *     other width (e.g. 44 columns), chosen per input.
+ *   - "[mxfp8 moe training] add bench script for scale conversion to blocked
+ *     format kernels for groups along K" (#3604): groups along K, each group
+ *     made of 128x4 scale-factor tiles.
+ *   - "Add CuTeDSL MXFP8 K-groups scale rearrange kernel" (#4704), review,
+ *     "Additional findings": padding is zero; empty groups add nothing; the
+ *     grid is over-provisioned by one chunk per group.
+ *
+ * Layout.  Scales are uint8 (E8M0), row-major (rows x cols) with a row
+ * stride in bytes; one scale per 32 data elements.  A group's padded matrix
+ * is cut into 128x4 tiles of 512 bytes, ordered row-block-major then
+ * column-block-minor; element (r, c) of a tile sits at byte
+ * (r%32)*16 + (r/32)*4 + c.
+ *   - Groups along M (forward / dgrad): group g is rows [E'[g-1], E'[g]),
+ *     padded to a multiple of 128 rows and roundup(cols, 4) columns; group g's
+ *     blocked rows start at row P_g = sum_{h<g} roundup(n_h, 128) of one
+ *     matrix roundup(cols, 4) wide.
+ *   - Groups along K (wgrad): group g is columns [E'[g-1], E'[g]), padded to
+ *     W_g = roundup(w_g, 4) columns and R = roundup(rows, 128) rows; group g's
+ *     blocked matrix (R x W_g) is stored contiguously at byte R * sum_{h<g} W_h.
+ *   Group ends E are int32 in device memory, cumulative (end of group g), in
+ *   rows (M) or scale columns (K).  They are read only on the device and are
+ *   clamped there, never rejected: E'[-1] = 0, E'[g] = min(max(E[g], E'[g-1]), T)
+ *   with T = rows (M) or cols (K).  Rows (M) or columns (K) past E'[G-1] are
+ *   ignored.  Every byte of the output allocation is written: real bytes,
+ *   zero padding, and a zero tail after the last group; the caller need not
+ *   clear `out`.
+ *
+ * Ownership and streams.  The caller owns every buffer.  The library never
+ * allocates, frees or synchronises, never reads device memory on the host,
+ * and launches only on `stream`, so every call may be captured in a CUDA
+ * graph (the pointers and shapes are then frozen into the graph).  The first
+ * call on a device sets kernel attributes and queries the device once; make
+ * that first call before any stream capture.  Calls are thread-safe.
+ *
+ * Errors.  Argument faults the host can see return a status and launch
+ * nothing.  A launch failure returns MX_ERR_CUDA (from cudaGetLastError).
+ * Bad device-side offsets are clamped as stated above.
+ */
+#ifndef MXSCALE_H
+#define MXSCALE_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MX_OK = 0,
+    MX_ERR_INVALID_ARG = 1,  /* null pointer, G outside [1, 64], negative size, stride < cols, sizes too large */
+    MX_ERR_MISALIGNED = 2,   /* `out` not 16-byte aligned, or a forced path whose alignment rule fails */
+    MX_ERR_UNSUPPORTED = 3,  /* shape beyond the kernels' index range */
+    MX_ERR_CUDA = 4          /* a CUDA runtime or driver call failed */
+} mx_status;
+
+typedef enum { MX_GROUPS_M = 0, MX_GROUPS_K = 1 } mx_group_dim;
+
+/* Kernel choice.  AUTO takes TMA when `scales` is 16-byte aligned and the
+ * row stride is a multiple of 16 bytes; otherwise WORD when both are
+ * multiples of 4; otherwise BYTE.  Forcing a path whose rule fails returns
+ * MX_ERR_MISALIGNED. */
+typedef enum { MX_PATH_AUTO = 0, MX_PATH_TMA = 1, MX_PATH_WORD = 2, MX_PATH_BYTE = 3 } mx_path;
+
+#define MX_MAX_GROUPS 64
+
+/* Bytes the caller must allocate for `out`:
+ *   M: (rows + 128 * num_groups) * roundup(cols, 4)
+ *   K: roundup(rows, 128) * (cols + 4 * num_groups)
+ * an upper bound on the padded output for any split of the groups, known on
+ * the host without reading the offsets.  Host-only.  Returns 0 for invalid
+ * arguments (and for shapes whose allocation is genuinely empty). */
+size_t mx_rearranged_size(mx_group_dim dim, int64_t rows, int64_t cols, int32_t num_groups);
+
+/* Groups along M.
+ *   scales             device, uint8, element (i, j) at scales[i * row_stride + j];
+ *                      any alignment; may be NULL when rows == 0 or cols == 0
+ *   rows, cols         >= 0, each at most 2^31 - 2^14
+ *   row_stride         bytes between rows, >= cols
+ *   group_end_offsets  device, int32[num_groups], cumulative row ends
+ *   num_groups         1..64
+ *   out                device, 16-byte aligned, mx_rearranged_size(MX_GROUPS_M, ...) bytes,
+ *                      must not overlap `scales`
+ *   stream             CUDA stream (0 = legacy default stream)
+ */
+mx_status mx_rearrange_m_groups(const uint8_t *scales, int64_t rows, int64_t cols, int64_t row_stride,
+                                const int32_t *group_end_offsets, int32_t num_groups, uint8_t *out,
+                                cudaStream_t stream);
+
+/* Groups along K: as mx_rearrange_m_groups, with group_end_offsets holding
+ * cumulative scale-column ends and `out` sized by mx_rearranged_size(MX_GROUPS_K, ...). */
+mx_status mx_rearrange_k_groups(const uint8_t *scales, int64_t rows, int64_t cols, int64_t row_stride,
+                                const int32_t *group_end_offsets, int32_t num_groups, uint8_t *out,
+                                cudaStream_t stream);
+
+/* Either dimension with an explicit kernel choice (tests and benchmarks). */
+mx_status mx_rearrange_ex(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t cols,
+                          int64_t row_stride, const int32_t *group_end_offsets, int32_t num_groups,
+                          uint8_t *out, mx_path path, cudaStream_t stream);
+
+/* The path AUTO would take for these arguments (host-only, no device access). */
+mx_path mx_select_path(mx_group_dim dim, const void *scales, int64_t rows, int64_t cols, int64_t row_stride);
+
+/* Static description of a status code. */
+const char *mx_status_string(mx_status status);
+
+/* Device-side error flags of the current device (bit 0: a pipeline wait ran
+ * past its time limit and the kernel returned early).  Synchronises the
+ * device: for tests and debugging, never on a hot path.  `clear` != 0 resets
+ * the flags after reading. */
+mx_status mx_device_flags(uint32_t *flags, int clear);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int mx_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MXSCALE_H */

@@ -1,1 +1,73 @@
-"""scale_factor_layout_b200: MXFP8 E8M0 scale factors -> per-group 128x4 blocked layout on B200."""
+"""scale_factor_layout_b200 -- MXFP8 E8M0 scale factors -> per-group 128x4
+blocked layout, on NVIDIA B200 (sm_100a).
+
+The work runs in libmxscale.so (C ABI in include/mxscale.h); this package is
+its binding.  ``_binding`` mirrors the C entry points one for one (raw
+pointers and sizes); the functions below take torch tensors for convenience,
+allocate the output with torch (the library itself never allocates), and pass
+torch's current CUDA stream.
+"""
+from __future__ import annotations
+
+from ._binding import (  # noqa: F401
+    MX_GROUPS_K, MX_GROUPS_M, MX_MAX_GROUPS, MX_OK, MX_PATH_AUTO, MX_PATH_BYTE, MX_PATH_TMA,
+    MX_PATH_WORD, PATHS, MxError, declared_symbols, lib, mx_device_flags, mx_rearrange_ex,
+    mx_rearrange_k_groups, mx_rearrange_m_groups, mx_rearranged_size, mx_select_path, mx_version,
+    status_string,
+)
+
+__all__ = [
+    "rearrange_m_groups", "rearrange_k_groups", "rearrange", "rearranged_size",
+    "mx_rearrange_m_groups", "mx_rearrange_k_groups", "mx_rearrange_ex", "mx_rearranged_size",
+    "mx_select_path", "mx_device_flags", "mx_version", "MxError",
+]
+
+
+def rearranged_size(dim: int, rows: int, cols: int, num_groups: int) -> int:
+    return mx_rearranged_size(dim, rows, cols, num_groups)
+
+
+def _check_inputs(scales, group_end_offsets):
+    import torch
+
+    if scales.dtype != torch.uint8 or scales.dim() != 2:
+        raise ValueError("scales must be a 2-D uint8 tensor")
+    if scales.shape[0] > 1 and scales.shape[1] > 1 and scales.stride(1) != 1:
+        raise ValueError("scales must be dense along columns (stride(1) == 1)")
+    if group_end_offsets.dtype != torch.int32 or group_end_offsets.dim() != 1:
+        raise ValueError("group_end_offsets must be a 1-D int32 tensor")
+    if not group_end_offsets.is_contiguous():
+        raise ValueError("group_end_offsets must be contiguous")
+    if not (scales.is_cuda and group_end_offsets.is_cuda):
+        raise ValueError("scales and group_end_offsets must be CUDA tensors")
+
+
+def rearrange(dim: int, scales, group_end_offsets, out=None, path: str = "auto", stream=None):
+    """Rearrange ``scales`` (rows, cols) uint8 for groups along M (dim 0) or K
+    (dim 1); returns the flat uint8 output of ``rearranged_size`` bytes."""
+    import torch
+
+    _check_inputs(scales, group_end_offsets)
+    rows, cols = scales.shape
+    G = group_end_offsets.numel()
+    size = mx_rearranged_size(dim, rows, cols, G)
+    if out is None:
+        out = torch.empty(size, dtype=torch.uint8, device=scales.device)
+    elif out.numel() < size or out.dtype != torch.uint8 or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous uint8 tensor of at least {size} bytes")
+    stride = scales.stride(0) if rows > 1 else cols
+    if stream is None:
+        stream = torch.cuda.current_stream(scales.device).cuda_stream
+    st = mx_rearrange_ex(dim, scales.data_ptr(), rows, cols, stride, group_end_offsets.data_ptr(), G,
+                         out.data_ptr(), PATHS[path], stream)
+    if st != MX_OK:
+        raise MxError("mx_rearrange_ex", st)
+    return out
+
+
+def rearrange_m_groups(scales, group_end_offsets, out=None, path: str = "auto"):
+    return rearrange(MX_GROUPS_M, scales, group_end_offsets, out, path)
+
+
+def rearrange_k_groups(scales, group_end_offsets, out=None, path: str = "auto"):
+    return rearrange(MX_GROUPS_K, scales, group_end_offsets, out, path)

@@ -1,0 +1,364 @@
+// mx_rearrange.cu -- libmxscale: MXFP8 E8M0 scale factors -> per-group 128x4
+// blocked layout on B200 (sm_100a).  Kernels and the C ABI of include/mxscale.h.
+//
+// Two kernels per grouping dimension:
+//   * rearrange_tma: persistent CTAs (one wave across the SMs); one thread
+//     streams 128-row boxes of scales into a ring of shared-memory stages with
+//     2-D TMA loads completed on mbarriers, while all 8 warps transpose the
+//     previous stages and store 512-byte tiles with 128-bit stores.  Needs the
+//     row stride to be a multiple of 16 bytes (the 2-D TMA stride rule named
+//     in pytorch/ao #3708, "fallback cuda kernel for when input doesn't meet
+//     2d TMA constraints", Context).
+//   * rearrange_fallback: the same work items loaded with ordinary 32-bit (or
+//     byte) loads, for any stride or alignment (#3708's fallback).
+// Every CTA scans the group ends itself (#3285, "compute prefix sum of group
+// sizes inside kernel", Changes), so no launch depends on device data known
+// to the host; the grid is sized from an upper bound on the work and CTAs
+// past the real work only help zero the allocation's tail (#4704 review,
+// "Grid over-provisioning" and "Output is torch.zeros every call").
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <mutex>
+
+#include "mx_device.cuh"
+#include "mxscale.h"
+
+namespace mx {
+
+// Error flags written by kernels (read back by mx_device_flags).
+__device__ unsigned int g_mx_flags = 0;
+
+constexpr int kStages = 4;
+
+template <bool kDimM>
+constexpr int stage_bytes() { return kDimM ? kStageBytesM : kStageBytesK; }
+
+template <bool kDimM>
+constexpr int tma_smem_bytes() { return kStages * stage_bytes<kDimM>() + 1024; }
+
+template <bool kDimM>
+__global__ void __launch_bounds__(kThreads)
+rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restrict__ ends,
+              uint8_t *__restrict__ out, int64_t out_size, Shape s) {
+    constexpr int kStageBytes = stage_bytes<kDimM>();
+    extern __shared__ uint8_t dyn_smem[];
+    // 128B swizzle needs 1024-byte aligned stage buffers
+    uint8_t *stages = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+    __shared__ GroupTable table;
+    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ Item items[kStages];
+
+    const int tid = threadIdx.x;
+    const int j = tid & 31;
+    const int q = tid >> 5;
+
+    if (tid == 0) {
+        tma_prefetch_desc(&tmap);
+#pragma unroll
+        for (int st = 0; st < kStages; ++st) mbar_init(&full[st], 1);
+        fence_mbar_init();
+    }
+    if (q == 0) build_group_table<kDimM>(ends, s.G, kDimM ? s.rows : s.cols, s.col_chunks, table);
+    __syncthreads();
+
+    const int total = total_items<kDimM>(table, s);
+    const int bid = blockIdx.x;
+    const int n_my = bid < total ? (total - 1 - bid) / (int)gridDim.x + 1 : 0;
+
+    auto issue = [&](int n, int st) {
+        const Item it = decode_item<kDimM>(table, s, bid + n * (int)gridDim.x, 16);
+        items[st] = it;
+        mbar_arrive_expect_tx(&full[st], kStageBytes);
+        tma_load_2d(stages + st * kStageBytes, &tmap, it.x, it.y, &full[st]);
+    };
+
+    if (tid == 0)
+        for (int st = 0; st < kStages && st < n_my; ++st) issue(st, st);
+
+    for (int n = 0; n < n_my; ++n) {
+        const int st = n % kStages;
+        const uint32_t parity = (uint32_t)(n / kStages) & 1u;
+        const bool ok = mbar_wait_bounded(&full[st], parity);
+        if (ok) {
+            const Item it = items[st];
+            const uint8_t *stage = stages + st * kStageBytes;
+            uint4 w[4];
+            if (kDimM)
+                read_rows_swizzled(stage, j, q, w);
+            else
+                read_rows_plain(stage, j, q, it.delta, w);
+            mask_and_store(w, it, j, q, out);
+        }
+        if (__syncthreads_or(!ok)) {
+            // A load never completed: flag it, wait (bounded) for the copies
+            // still in flight into this CTA's shared memory, and leave.
+            if (tid == 0) {
+                atomicOr(&g_mx_flags, kFlagWaitTimeout);
+                for (int m = n; m < n_my && m < n + kStages; ++m)
+                    mbar_wait_bounded(&full[m % kStages], (uint32_t)(m / kStages) & 1u);
+            }
+            return;
+        }
+        if (tid == 0 && n + kStages < n_my) {
+            fence_proxy_async_smem();
+            issue(n + kStages, st);
+        }
+    }
+    zero_tail(out, covered_bytes<kDimM>(table, s), out_size);
+}
+
+template <bool kDimM, bool kWord>
+__global__ void __launch_bounds__(kThreads)
+rearrange_fallback(const uint8_t *__restrict__ scales, int64_t row_stride, const int32_t *__restrict__ ends,
+                   uint8_t *__restrict__ out, int64_t out_size, Shape s) {
+    __shared__ __align__(16) uint8_t stage[kStageBytesK];
+    __shared__ GroupTable table;
+    const int tid = threadIdx.x;
+    const int j = tid & 31;
+    const int q = tid >> 5;
+
+    if (q == 0) build_group_table<kDimM>(ends, s.G, kDimM ? s.rows : s.cols, s.col_chunks, table);
+    __syncthreads();
+    const int total = total_items<kDimM>(table, s);
+
+    for (int i = blockIdx.x; i < total; i += gridDim.x) {
+        const Item it = decode_item<kDimM>(table, s, i, kWord ? 4 : 1);
+        // stage row r holds the chunk's bytes from column it.x on
+        const int nw = (it.delta + it.cols_valid + 3) >> 2;
+        const int nwords = it.rows_valid * nw;
+        for (int idx = tid; idx < nwords; idx += kThreads) {
+            const int r = idx / nw;
+            const int w = idx - r * nw;
+            const int gcol = it.x + 4 * w;
+            const uint8_t *src = scales + (int64_t)(it.y + r) * row_stride + gcol;
+            uint32_t v;
+            if (kWord && gcol + 4 <= s.cols) {
+                v = __ldg(reinterpret_cast<const uint32_t *>(src));
+            } else {
+                v = 0;
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    if (gcol + b < s.cols) v |= (uint32_t)__ldg(src + b) << (8 * b);
+            }
+            *reinterpret_cast<uint32_t *>(stage + r * kPitchPlain + 4 * w) = v;
+        }
+        __syncthreads();
+        uint4 w4[4];
+        read_rows_plain(stage, j, q, it.delta, w4);
+        mask_and_store(w4, it, j, q, out);
+        __syncthreads();
+    }
+    zero_tail(out, covered_bytes<kDimM>(table, s), out_size);
+}
+
+// ------------------------------------------------------------------ host side
+constexpr int64_t kMaxExtent = (1ll << 31) - (1ll << 14);
+constexpr int kMaxDevices = 128;
+
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+    int occ_tma[2] = {0, 0};   // [dimM]
+    int occ_fallback = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode;
+}
+
+mx_status device_info(const DeviceInfo **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MX_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MX_ERR_CUDA;
+        if (cudaFuncSetAttribute(rearrange_tma<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tma_smem_bytes<true>()) != cudaSuccess ||
+            cudaFuncSetAttribute(rearrange_tma<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tma_smem_bytes<false>()) != cudaSuccess)
+            return MX_ERR_CUDA;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_tma[1], rearrange_tma<true>, kThreads,
+                                                          tma_smem_bytes<true>()) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_tma[0], rearrange_tma<false>, kThreads,
+                                                          tma_smem_bytes<false>()) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_fallback, rearrange_fallback<true, true>,
+                                                          kThreads, 0) != cudaSuccess)
+            return MX_ERR_CUDA;
+        if (d.occ_tma[0] < 1 || d.occ_tma[1] < 1 || d.occ_fallback < 1) return MX_ERR_CUDA;
+        d.ready = true;
+    }
+    *out = &d;
+    return MX_OK;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+bool tma_eligible(const void *scales, int64_t rows, int64_t cols, int64_t row_stride) {
+    return rows >= 1 && cols >= 1 && (reinterpret_cast<uintptr_t>(scales) & 15u) == 0 &&
+           (row_stride & 15) == 0 && row_stride < (1ll << 40);
+}
+
+bool word_eligible(const void *scales, int64_t row_stride) {
+    return (reinterpret_cast<uintptr_t>(scales) & 3u) == 0 && (row_stride & 3) == 0;
+}
+
+mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t cols, int64_t row_stride,
+              const int32_t *ends, int32_t G, uint8_t *out, mx_path path, cudaStream_t stream) {
+    if (dim != MX_GROUPS_M && dim != MX_GROUPS_K) return MX_ERR_INVALID_ARG;
+    if (path < MX_PATH_AUTO || path > MX_PATH_BYTE) return MX_ERR_INVALID_ARG;
+    if (G < 1 || G > MX_MAX_GROUPS) return MX_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || rows > kMaxExtent || cols > kMaxExtent) return MX_ERR_INVALID_ARG;
+    if (row_stride < cols) return MX_ERR_INVALID_ARG;
+    if (ends == nullptr) return MX_ERR_INVALID_ARG;
+    const bool dim_m = dim == MX_GROUPS_M;
+    const size_t size = mx_rearranged_size(dim, rows, cols, G);
+    if (size > 0 && out == nullptr) return MX_ERR_INVALID_ARG;
+    if (rows > 0 && cols > 0 && scales == nullptr) return MX_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(out) & 15u) != 0) return MX_ERR_MISALIGNED;
+    if (size == 0) return MX_OK;
+
+    Shape s;
+    s.rows = (int32_t)rows;
+    s.cols = (int32_t)cols;
+    s.G = G;
+    s.padded_cols = (int32_t)round_up(cols, 4);
+    s.padded_rows = (int32_t)round_up(rows, 128);
+    s.col_chunks = (int32_t)ceil_div(s.padded_cols, kChunkCols);
+    // Upper bound on work items, known without reading the offsets.
+    const int64_t bound = dim_m ? (ceil_div(rows, 128) + G) * s.col_chunks
+                                : ceil_div(rows, 128) * (ceil_div(cols, kChunkCols) + G);
+    if (bound > INT_MAX) return MX_ERR_UNSUPPORTED;
+
+    const bool degenerate = rows == 0 || cols == 0;
+    if (path == MX_PATH_AUTO)
+        path = tma_eligible(scales, rows, cols, row_stride) ? MX_PATH_TMA
+               : word_eligible(scales, row_stride)          ? MX_PATH_WORD
+                                                            : MX_PATH_BYTE;
+    if (degenerate) path = MX_PATH_WORD;  // nothing to load: only the zero fill runs
+    if (path == MX_PATH_TMA && !tma_eligible(scales, rows, cols, row_stride)) return MX_ERR_MISALIGNED;
+    if (path == MX_PATH_WORD && !degenerate && !word_eligible(scales, row_stride)) return MX_ERR_MISALIGNED;
+
+    const DeviceInfo *d = nullptr;
+    if (mx_status st = device_info(&d); st != MX_OK) return st;
+    const int64_t work = bound > 0 ? bound : 1;
+
+    if (path == MX_PATH_TMA) {
+        auto encode = encode_fn();
+        if (encode == nullptr) return MX_ERR_CUDA;
+        CUtensorMap map;
+        cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+        cuuint64_t gstride[1] = {(cuuint64_t)row_stride};
+        cuuint32_t box[2] = {(cuuint32_t)(dim_m ? kPitchSw : kPitchPlain), (cuuint32_t)kTileRows};
+        cuuint32_t estride[2] = {1, 1};
+        CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(scales), gdim, gstride,
+                            box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            dim_m ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return MX_ERR_CUDA;
+        const int64_t cap = (int64_t)d->sms * d->occ_tma[dim_m ? 1 : 0];
+        const int grid = (int)(work < cap ? work : cap);
+        if (dim_m)
+            rearrange_tma<true><<<grid, kThreads, tma_smem_bytes<true>(), stream>>>(map, ends, out, (int64_t)size, s);
+        else
+            rearrange_tma<false><<<grid, kThreads, tma_smem_bytes<false>(), stream>>>(map, ends, out, (int64_t)size, s);
+    } else {
+        const int64_t cap = (int64_t)d->sms * d->occ_fallback * 4;
+        const int grid = (int)(work < cap ? work : cap);
+        const bool word = path == MX_PATH_WORD;
+        if (dim_m && word)
+            rearrange_fallback<true, true><<<grid, kThreads, 0, stream>>>(scales, row_stride, ends, out, (int64_t)size, s);
+        else if (dim_m)
+            rearrange_fallback<true, false><<<grid, kThreads, 0, stream>>>(scales, row_stride, ends, out, (int64_t)size, s);
+        else if (word)
+            rearrange_fallback<false, true><<<grid, kThreads, 0, stream>>>(scales, row_stride, ends, out, (int64_t)size, s);
+        else
+            rearrange_fallback<false, false><<<grid, kThreads, 0, stream>>>(scales, row_stride, ends, out, (int64_t)size, s);
+    }
+    return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
+}  // namespace mx
+
+// ------------------------------------------------------------------ C ABI
+extern "C" {
+
+size_t mx_rearranged_size(mx_group_dim dim, int64_t rows, int64_t cols, int32_t num_groups) {
+    if ((dim != MX_GROUPS_M && dim != MX_GROUPS_K) || rows < 0 || cols < 0 || num_groups < 1 ||
+        num_groups > MX_MAX_GROUPS || rows > mx::kMaxExtent || cols > mx::kMaxExtent)
+        return 0;
+    if (dim == MX_GROUPS_M) return (size_t)((rows + 128ll * num_groups) * mx::round_up(cols, 4));
+    return (size_t)(mx::round_up(rows, 128) * (cols + 4ll * num_groups));
+}
+
+mx_status mx_rearrange_m_groups(const uint8_t *scales, int64_t rows, int64_t cols, int64_t row_stride,
+                                const int32_t *group_end_offsets, int32_t num_groups, uint8_t *out,
+                                cudaStream_t stream) {
+    return mx::run(MX_GROUPS_M, scales, rows, cols, row_stride, group_end_offsets, num_groups, out,
+                   MX_PATH_AUTO, stream);
+}
+
+mx_status mx_rearrange_k_groups(const uint8_t *scales, int64_t rows, int64_t cols, int64_t row_stride,
+                                const int32_t *group_end_offsets, int32_t num_groups, uint8_t *out,
+                                cudaStream_t stream) {
+    return mx::run(MX_GROUPS_K, scales, rows, cols, row_stride, group_end_offsets, num_groups, out,
+                   MX_PATH_AUTO, stream);
+}
+
+mx_status mx_rearrange_ex(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t cols,
+                          int64_t row_stride, const int32_t *group_end_offsets, int32_t num_groups,
+                          uint8_t *out, mx_path path, cudaStream_t stream) {
+    return mx::run(dim, scales, rows, cols, row_stride, group_end_offsets, num_groups, out, path, stream);
+}
+
+mx_path mx_select_path(mx_group_dim dim, const void *scales, int64_t rows, int64_t cols, int64_t row_stride) {
+    (void)dim;
+    if (mx::tma_eligible(scales, rows, cols, row_stride)) return MX_PATH_TMA;
+    if (mx::word_eligible(scales, row_stride) || rows == 0 || cols == 0) return MX_PATH_WORD;
+    return MX_PATH_BYTE;
+}
+
+const char *mx_status_string(mx_status status) {
+    switch (status) {
+        case MX_OK: return "ok";
+        case MX_ERR_INVALID_ARG: return "invalid argument";
+        case MX_ERR_MISALIGNED: return "misaligned pointer or stride for the requested path";
+        case MX_ERR_UNSUPPORTED: return "shape beyond the supported index range";
+        case MX_ERR_CUDA: return "CUDA call failed";
+    }
+    return "unknown status";
+}
+
+mx_status mx_device_flags(uint32_t *flags, int clear) {
+    if (flags == nullptr) return MX_ERR_INVALID_ARG;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, mx::g_mx_flags, sizeof(v)) != cudaSuccess) return MX_ERR_CUDA;
+    *flags = v;
+    if (clear) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(mx::g_mx_flags, &zero, sizeof(zero)) != cudaSuccess) return MX_ERR_CUDA;
+    }
+    return MX_OK;
+}
+
+int mx_version(void) { return 100; }
+
+}  // extern "C"

@@ -18,3 +18,21 @@ def orc():
 
     oracle.load()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def mxlib():
+    """libmxscale built in-tree (nvcc cross-compiles without a GPU)."""
+    from scale_factor_layout_b200 import _build, _binding
+
+    _build.build()
+    return _binding.lib()
+
+
+def gpu_available():
+    try:
+        import torch
+
+        return torch.cuda.is_available()
+    except Exception:
+        return False

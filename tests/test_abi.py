@@ -1,0 +1,72 @@
+"""C ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, sizes outputs like the oracle, picks paths by the stated
+alignment rules, and rejects bad arguments before touching the device."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from scale_factor_layout_b200 import _binding as B
+
+M, K = B.MX_GROUPS_M, B.MX_GROUPS_K
+
+
+def test_exports_every_declared_symbol(mxlib):
+    declared = B.declared_symbols()
+    assert {"mx_rearrange_m_groups", "mx_rearrange_k_groups", "mx_rearranged_size"} <= set(declared)
+    for name in declared:
+        assert hasattr(mxlib, name), f"{name} declared in include/mxscale.h but not exported"
+    assert B.mx_version() >= 100
+
+
+def test_sizes_match_oracle(mxlib, orc):
+    rng = np.random.default_rng(0)
+    for _ in range(500):
+        dim = int(rng.integers(0, 2))
+        rows, cols, G = int(rng.integers(0, 300000)), int(rng.integers(0, 20000)), int(rng.integers(1, 65))
+        assert B.mx_rearranged_size(dim, rows, cols, G) == orc.rearranged_size(dim, rows, cols, G)
+    for bad in ((M, 10, 10, 0), (M, 10, 10, 65), (K, -1, 10, 1), (K, 10, -1, 1), (2, 10, 10, 1)):
+        assert B.mx_rearranged_size(*bad) == 0
+
+
+def test_path_selection(mxlib):
+    assert B.mx_select_path(M, 0x1000, 100, 224, 224) == B.MX_PATH_TMA
+    assert B.mx_select_path(M, 0x1000, 100, 44, 44) == B.MX_PATH_WORD
+    assert B.mx_select_path(M, 0x1004, 100, 48, 48) == B.MX_PATH_WORD      # base not 16-aligned
+    assert B.mx_select_path(K, 0x1000, 100, 45, 45) == B.MX_PATH_BYTE      # odd stride
+    assert B.mx_select_path(K, 0x1001, 100, 48, 48) == B.MX_PATH_BYTE      # odd base
+    assert B.mx_select_path(K, 0x1000, 7168, 4096, 4096) == B.MX_PATH_TMA
+    assert B.mx_select_path(K, 0x1000, 0, 4096, 4096) == B.MX_PATH_WORD    # nothing to load
+
+
+def _call(dim=M, scales=0x1000, rows=256, cols=64, stride=64, ends=0x2000, G=2, out=0x3000, path=0):
+    return B.mx_rearrange_ex(dim, scales, rows, cols, stride, ends, G, out, path, 0)
+
+
+@pytest.mark.parametrize("kwargs,status", [
+    (dict(G=0), B.MX_ERR_INVALID_ARG),
+    (dict(G=65), B.MX_ERR_INVALID_ARG),
+    (dict(rows=-1), B.MX_ERR_INVALID_ARG),
+    (dict(cols=-5), B.MX_ERR_INVALID_ARG),
+    (dict(rows=1 << 31), B.MX_ERR_INVALID_ARG),
+    (dict(stride=63), B.MX_ERR_INVALID_ARG),
+    (dict(ends=0), B.MX_ERR_INVALID_ARG),
+    (dict(out=0), B.MX_ERR_INVALID_ARG),
+    (dict(scales=0), B.MX_ERR_INVALID_ARG),
+    (dict(dim=3), B.MX_ERR_INVALID_ARG),
+    (dict(path=7), B.MX_ERR_INVALID_ARG),
+    (dict(out=0x3008), B.MX_ERR_MISALIGNED),
+    (dict(stride=72, path=B.MX_PATH_TMA), B.MX_ERR_MISALIGNED),
+    (dict(scales=0x1008, path=B.MX_PATH_TMA), B.MX_ERR_MISALIGNED),
+    (dict(stride=66, path=B.MX_PATH_WORD), B.MX_ERR_MISALIGNED),
+    (dict(scales=0x1002, path=B.MX_PATH_WORD), B.MX_ERR_MISALIGNED),
+    (dict(dim=K, rows=0), B.MX_OK),          # empty allocation: nothing to do, no launch
+])
+def test_host_validation(mxlib, kwargs, status):
+    assert _call(**kwargs) == status
+
+
+def test_status_strings(mxlib):
+    for st in range(5):
+        assert B.status_string(st)
+    assert "misaligned" in B.status_string(B.MX_ERR_MISALIGNED)
