@@ -10,11 +10,12 @@ Metric: GB/s = (bytes of real scales read + exact padded bytes written) / time,
 and the same as a fraction of the measured HBM copy bandwidth.
 
 Timing: the K timed steps are captured in one CUDA graph (as the pages timed
-their kernels) and replayed once between CUDA events; inputs and outputs
+their kernels) and replayed once between two CUDA events; inputs and outputs
 rotate over enough buffer sets that one rotation spans more than 4x the L2,
-so every step reads cold inputs.  Timing events captured inside the graph
-give each kernel's own duration.  Multi-GPU: independent replicas, one
-process per GPU (torchrun), max time over ranks.
+so every step reads cold inputs.  Each call's own duration comes from a
+second graph per call type: the same K launches of that call, back to back,
+between two CUDA events.  Multi-GPU: independent replicas, one process per
+GPU (torchrun), max time over ranks.
 
 --impl reference times the CPU oracle (the plain C statement of the layout)
 on this host on a bounded sample of the same workload.
@@ -228,24 +229,26 @@ def aggregate_value(bytes_per_step: int, steps: int, n_gpus: int, seconds: float
 
 
 # ------------------------------------------------------------------ GPU arm
-class DeviceSet:
-    """One rotation set: device copies of every case's inputs plus outputs."""
+def device_copies(case, n, device):
+    """n independent device copies of a case's inputs, each with its own output."""
+    import torch
 
-    def __init__(self, cases, device):
-        import torch
+    import scale_factor_layout_b200 as mxs
 
-        import scale_factor_layout_b200 as mxs
+    out = []
+    host_s = torch.from_numpy(np.ascontiguousarray(case.scales))
+    host_e = torch.from_numpy(np.ascontiguousarray(case.ends, dtype=np.int32))
+    size = mxs.mx_rearranged_size(case.dim, case.rows, case.cols, case.num_groups)
+    for _ in range(n):
+        out.append((case, host_s.to(device), host_e.to(device),
+                    torch.empty(size, dtype=torch.uint8, device=device)))
+    return out
 
-        self.items = []
-        for c in cases:
-            s = torch.from_numpy(np.ascontiguousarray(c.scales)).to(device)
-            e = torch.from_numpy(np.ascontiguousarray(c.ends, dtype=np.int32)).to(device)
-            size = mxs.mx_rearranged_size(c.dim, c.rows, c.cols, c.num_groups)
-            o = torch.empty(size, dtype=torch.uint8, device=device)
-            self.items.append((c, s, e, o))
 
-    def bytes(self):
-        return sum(i[1].numel() + i[3].numel() for i in self.items)
+def rotation_count(case) -> int:
+    """Copies needed so that one rotation of this call alone spans 4x the L2."""
+    b = algorithmic_bytes(case)
+    return max(2, math.ceil(4 * L2_BYTES / (b["read"] + b["alloc"])))
 
 
 def launch(item, stream_handle):
@@ -273,72 +276,75 @@ def run_ours(args, rank, world, local):
     step_bytes = sum(b["read"] + b["written"] for b in per_call)
     step_bytes_pages = sum(b["read"] + b["alloc"] for b in per_call)
 
-    first = DeviceSet(cases, device)
-    n_sets = max(2, math.ceil(4 * L2_BYTES / first.bytes()))
-    sets = [first] + [DeviceSet(cases, device) for _ in range(n_sets - 1)]
+    rot = [device_copies(c, rotation_count(c), device) for c in cases]
+    rot_bytes = sum(len(r) * (algorithmic_bytes(c)["read"] + algorithmic_bytes(c)["alloc"])
+                    for c, r in zip(cases, rot))
     stream = torch.cuda.Stream(device)
     h = stream.cuda_stream
     ncalls = len(cases)
+
+    def step_items(k):
+        return [r[k % len(r)] for r in rot]
+
     with torch.cuda.stream(stream):
         for k in range(3):  # first calls set kernel attributes (outside capture) and warm caches
-            for it in sets[k % n_sets].items:
+            for it in step_items(k):
                 launch(it, h)
     torch.cuda.synchronize()
 
-    def capture(steps, with_events):
+    def capture(launches):
+        """One CUDA graph holding the given (item) launches back to back."""
         g = torch.cuda.CUDAGraph()
-        evs = []
         with torch.cuda.stream(stream):
             with torch.cuda.graph(g, stream=stream):
-                for k in range(steps):
-                    row = []
-                    for it in sets[k % n_sets].items:
-                        if with_events:
-                            ev = torch.cuda.Event(enable_timing=True, external=True)
-                            ev.record(stream)
-                            row.append(ev)
-                        launch(it, h)
-                    if with_events:
-                        ev = torch.cuda.Event(enable_timing=True, external=True)
-                        ev.record(stream)
-                        row.append(ev)
-                    evs.append(row)
-        return g, evs
+                for it in launches:
+                    launch(it, h)
+        return g
 
-    warm_g, _ = capture(args.warmup, False)
-    timed_g, evs = capture(args.steps, True)
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
+    def steps_of(k0, n):
+        return [it for k in range(k0, k0 + n) for it in step_items(k)]
+
+    def replay_timed(g):
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier(dist, device)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            g.replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+        barrier(dist, device)
+        return start.elapsed_time(end) / 1e3
+
+    warm_g = capture(steps_of(0, args.warmup))
+    timed_g = capture(steps_of(args.warmup, args.steps))
+    # each call on its own: the same launches back to back, one call type per graph
+    per_call_g = [capture([rot[i][k % len(rot[i])] for k in range(args.steps)]) for i in range(ncalls)]
 
     sampler = ClockSampler(local)
     with sampler:
         with torch.cuda.stream(stream):
             warm_g.replay()
-        torch.cuda.synchronize()
-        barrier(dist, device)
-        torch.cuda.synchronize()
         t0 = time.perf_counter()
-        with torch.cuda.stream(stream):
-            start.record(stream)
-            timed_g.replay()
-            end.record(stream)
-        torch.cuda.synchronize()
+        seconds = replay_timed(timed_g)
         t1 = time.perf_counter()
-        barrier(dist, device)
         sampler.window = (t0, t1)
-    seconds = start.elapsed_time(end) / 1e3
+        avg = []
+        for g in per_call_g:
+            with torch.cuda.stream(stream):
+                warm_g.replay()
+            avg.append(max_over_ranks(replay_timed(g), dist, device) / args.steps)
     seconds_max = max_over_ranks(seconds, dist, device)
-    # per-kernel durations from the events captured around each call
-    durs = [[r[i].elapsed_time(r[i + 1]) / 1e3 for r in evs] for i in range(ncalls)]
-    avg = [statistics.fmean(d) for d in durs]
-    del timed_g, warm_g
+    del timed_g, warm_g, per_call_g
 
     peak, peak_src = load_peaks()
     value = aggregate_value(step_bytes, args.steps, world, seconds_max)
     calls = []
     for c, b, t in zip(cases, per_call, avg):
         gbs = (b["read"] + b["written"]) / t / 1e9
-        path = mxs.mx_select_path(c.dim, sets[0].items[cases.index(c)][1].data_ptr(), c.rows, c.cols, c.cols)
+        path = mxs.mx_select_path(c.dim, rot[cases.index(c)][0][1].data_ptr(), c.rows, c.cols, c.cols)
         calls.append({"case": c.name, "path": {1: "tma", 2: "word", 3: "byte"}.get(path, "?"),
                       "us": round(t * 1e6, 3), "gbps": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
                       "read_bytes": b["read"], "written_bytes": b["written"], "alloc_bytes": b["alloc"],
@@ -361,8 +367,10 @@ def run_ours(args, rank, world, local):
         "config": {"workload": args.workload, "description": WORKLOAD_DESC[args.workload],
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "bytes_per_step": step_bytes, "bytes_per_step_pages_convention": step_bytes_pages,
-                   "l2": f"rotating {n_sets} input/output sets, {n_sets * first.bytes() / 1e6:.0f} MB > 4x L2",
-                   "timing": "one CUDA graph of all timed steps, CUDA events, max over ranks"},
+                   "l2": "inputs/outputs rotate per call over " + ", ".join(str(len(r)) for r in rot)
+                         + f" copies ({rot_bytes / 1e6:.0f} MB); each call's rotation alone spans > 4x L2",
+                   "timing": "one CUDA graph of all timed steps between two CUDA events, max over ranks; "
+                             "per-call durations from one graph per call type (same launches, back to back)"},
         "frac_of_peak": round(value / world / peak, 4),
         "calls": calls,
         "roofline": roofline,

@@ -84,6 +84,30 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
+// Bulk asynchronous shared -> global copy (bytes a multiple of 16, both
+// addresses 16-byte aligned), tracked per issuing thread in bulk groups.
+__device__ __forceinline__ void bulk_store_s2g(void *gdst, const void *ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(gdst)), "r"(smem_addr(ssrc)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until all of this thread's bulk groups have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Programmatic dependent launch: wait for the grids this launch depends on
+// (a no-op when launched without the attribute), and allow dependents to be
+// scheduled.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ scan
 // Per-group values every CTA derives from the raw end offsets.
 struct GroupTable {
@@ -325,6 +349,29 @@ __device__ __forceinline__ void mask_and_store(const uint4 (&w)[4], const Item &
             o.z = word_of(w[2], t) & rm[2] & cm;
             o.w = word_of(w[3], t) & rm[3] & cm;
             *reinterpret_cast<uint4 *>(base + (int64_t)tile * 512) = o;
+        }
+    }
+}
+
+// As mask_and_store, but into a shared-memory staging block laid out exactly
+// like the item's output span (tile t at byte 512 t), for a bulk store.
+__device__ __forceinline__ void mask_and_stage(const uint4 (&w)[4], const Item &it, int j, int q,
+                                               uint8_t *staging) {
+    uint32_t rm[4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) rm[a] = (j + 32 * a < it.rows_valid) ? 0xffffffffu : 0u;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int tile = 4 * q + t;
+        if (tile < it.ntiles) {
+            const int nv = it.cols_valid - 4 * tile;
+            const uint32_t cm = nv >= 4 ? 0xffffffffu : (nv <= 0 ? 0u : ((1u << (8 * nv)) - 1u));
+            uint4 o;
+            o.x = word_of(w[0], t) & rm[0] & cm;
+            o.y = word_of(w[1], t) & rm[1] & cm;
+            o.z = word_of(w[2], t) & rm[2] & cm;
+            o.w = word_of(w[3], t) & rm[3] & cm;
+            *reinterpret_cast<uint4 *>(staging + tile * 512 + 16 * j) = o;
         }
     }
 }

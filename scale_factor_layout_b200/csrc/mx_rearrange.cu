@@ -32,16 +32,28 @@ namespace mx {
 // Error flags written by kernels (read back by mx_device_flags).
 __device__ unsigned int g_mx_flags = 0;
 
-constexpr int kStages = 4;
+constexpr int kStages = 4;       // input boxes in flight per CTA
+constexpr int kOutBuffers = 2;   // output staging blocks per CTA
+constexpr int kOutBytes = kTilesPerChunk * 512;
 
 template <bool kDimM>
 constexpr int stage_bytes() { return kDimM ? kStageBytesM : kStageBytesK; }
 
 template <bool kDimM>
-constexpr int tma_smem_bytes() { return kStages * stage_bytes<kDimM>() + 1024; }
+constexpr int tma_smem_bytes() { return kStages * stage_bytes<kDimM>() + kOutBuffers * kOutBytes + 1024; }
 
+// Persistent TMA kernel.  Per work item n of this CTA:
+//   1. wait for its input box (stage n % kStages) and read 4 rows x 16 bytes
+//      per thread into registers;
+//   2. one barrier: the stage and the staging block n % 2 are free, and the
+//      staging block of item n-1 is complete;
+//   3. thread 0 bulk-stores item n-1's tiles (shared -> global, asynchronous)
+//      and refills the stage with the TMA load of item n + kStages;
+//   4. every thread writes its masked output lines of item n into staging.
+// Loads and stores are both asynchronous copies driven by one thread, so the
+// 8 warps only move data between shared memory and registers.
 template <bool kDimM>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restrict__ ends,
               uint8_t *__restrict__ out, int64_t out_size, Shape s) {
     constexpr int kStageBytes = stage_bytes<kDimM>();
@@ -49,6 +61,7 @@ rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restric
     // 128B swizzle needs 1024-byte aligned stage buffers
     uint8_t *stages = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+    uint8_t *staging = stages + kStages * kStageBytes;
     __shared__ GroupTable table;
     __shared__ __align__(8) uint64_t full[kStages];
     __shared__ Item items[kStages];
@@ -63,8 +76,12 @@ rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restric
         for (int st = 0; st < kStages; ++st) mbar_init(&full[st], 1);
         fence_mbar_init();
     }
+    // Inputs may come from the previous kernel in the stream; outputs may
+    // still be read by it.  Nothing global is touched before this point.
+    grid_dependency_wait();
     if (q == 0) build_group_table<kDimM>(ends, s.G, kDimM ? s.rows : s.cols, s.col_chunks, table);
     __syncthreads();
+    grid_launch_dependents();
 
     const int total = total_items<kDimM>(table, s);
     const int bid = blockIdx.x;
@@ -80,20 +97,25 @@ rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restric
     if (tid == 0)
         for (int st = 0; st < kStages && st < n_my; ++st) issue(st, st);
 
+    int64_t prev_off = 0;     // thread 0: output span of the previous item
+    uint32_t prev_bytes = 0;
     for (int n = 0; n < n_my; ++n) {
         const int st = n % kStages;
         const uint32_t parity = (uint32_t)(n / kStages) & 1u;
         const bool ok = mbar_wait_bounded(&full[st], parity);
+        uint4 w[4];
+        Item it;
         if (ok) {
-            const Item it = items[st];
+            it = items[st];
             const uint8_t *stage = stages + st * kStageBytes;
-            uint4 w[4];
             if (kDimM)
                 read_rows_swizzled(stage, j, q, w);
             else
                 read_rows_plain(stage, j, q, it.delta, w);
-            mask_and_store(w, it, j, q, out);
         }
+        // the store that last read staging block n % 2 (item n-2) is the only
+        // bulk group still outstanding here
+        if (tid == 0) bulk_wait_read<0>();
         if (__syncthreads_or(!ok)) {
             // A load never completed: flag it, wait (bounded) for the copies
             // still in flight into this CTA's shared memory, and leave.
@@ -104,13 +126,35 @@ rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restric
             }
             return;
         }
-        if (tid == 0 && n + kStages < n_my) {
-            fence_proxy_async_smem();
-            issue(n + kStages, st);
+        if (tid == 0) {
+            if (n > 0) {
+                bulk_store_s2g(out + prev_off, staging + ((n - 1) & 1) * kOutBytes, prev_bytes);
+                bulk_commit();
+            }
+            prev_off = it.out_off;
+            prev_bytes = (uint32_t)it.ntiles * 512u;
+            if (n + kStages < n_my) issue(n + kStages, st);
+        }
+        mask_and_stage(w, it, j, q, staging + (n & 1) * kOutBytes);
+        fence_proxy_async_smem();
+    }
+    if (n_my > 0) {
+        __syncthreads();
+        if (tid == 0) {
+            bulk_store_s2g(out + prev_off, staging + ((n_my - 1) & 1) * kOutBytes, prev_bytes);
+            bulk_commit();
         }
     }
     zero_tail(out, covered_bytes<kDimM>(table, s), out_size);
+    if (tid == 0) bulk_wait_all();
 }
+
+// Fallback for any stride and alignment.  One work item per loop trip: every
+// thread first issues all of its loads for the item (up to kMaxWordsPerThread
+// 32-bit words, or their bytes), then parks them in shared memory; the
+// transpose and stores match the TMA kernel's.
+constexpr int kMaxWordsPerRow = (3 + kChunkCols + 3) / 4;   // chunk may start 3 bytes into a word
+constexpr int kMaxWordsPerThread = (kTileRows * kMaxWordsPerRow + kThreads - 1) / kThreads;
 
 template <bool kDimM, bool kWord>
 __global__ void __launch_bounds__(kThreads)
@@ -122,30 +166,48 @@ rearrange_fallback(const uint8_t *__restrict__ scales, int64_t row_stride, const
     const int j = tid & 31;
     const int q = tid >> 5;
 
+    grid_dependency_wait();
     if (q == 0) build_group_table<kDimM>(ends, s.G, kDimM ? s.rows : s.cols, s.col_chunks, table);
     __syncthreads();
     const int total = total_items<kDimM>(table, s);
 
     for (int i = blockIdx.x; i < total; i += gridDim.x) {
         const Item it = decode_item<kDimM>(table, s, i, kWord ? 4 : 1);
-        // stage row r holds the chunk's bytes from column it.x on
+        // stage row r holds the chunk's bytes from column it.x on, in words
         const int nw = (it.delta + it.cols_valid + 3) >> 2;
-        const int nwords = it.rows_valid * nw;
-        for (int idx = tid; idx < nwords; idx += kThreads) {
-            const int r = idx / nw;
-            const int w = idx - r * nw;
-            const int gcol = it.x + 4 * w;
-            const uint8_t *src = scales + (int64_t)(it.y + r) * row_stride + gcol;
-            uint32_t v;
-            if (kWord && gcol + 4 <= s.cols) {
-                v = __ldg(reinterpret_cast<const uint32_t *>(src));
-            } else {
-                v = 0;
+        const int dr = kThreads / nw, dw = kThreads - dr * nw;   // (row, word) step per trip
+        const int r0 = tid / nw, w0 = tid - r0 * nw;
+        uint32_t v[kMaxWordsPerThread];
+        {
+            int r = r0, w = w0;
 #pragma unroll
-                for (int b = 0; b < 4; ++b)
-                    if (gcol + b < s.cols) v |= (uint32_t)__ldg(src + b) << (8 * b);
+            for (int u = 0; u < kMaxWordsPerThread; ++u) {
+                v[u] = 0;
+                if (r < it.rows_valid) {
+                    const int gcol = it.x + 4 * w;
+                    const uint8_t *src = scales + (int64_t)(it.y + r) * row_stride + gcol;
+                    if (kWord && gcol + 4 <= s.cols) {
+                        v[u] = __ldg(reinterpret_cast<const uint32_t *>(src));
+                    } else {
+#pragma unroll
+                        for (int b = 0; b < 4; ++b)
+                            if (gcol + b < s.cols) v[u] |= (uint32_t)__ldg(src + b) << (8 * b);
+                    }
+                }
+                r += dr;
+                w += dw;
+                if (w >= nw) { w -= nw; ++r; }
             }
-            *reinterpret_cast<uint32_t *>(stage + r * kPitchPlain + 4 * w) = v;
+        }
+        {
+            int r = r0, w = w0;
+#pragma unroll
+            for (int u = 0; u < kMaxWordsPerThread; ++u) {
+                if (r < it.rows_valid) *reinterpret_cast<uint32_t *>(stage + r * kPitchPlain + 4 * w) = v[u];
+                r += dr;
+                w += dw;
+                if (w >= nw) { w -= nw; ++r; }
+            }
         }
         __syncthreads();
         uint4 w4[4];
@@ -207,6 +269,24 @@ mx_status device_info(const DeviceInfo **out) {
     }
     *out = &d;
     return MX_OK;
+}
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream drains; it waits for that kernel's
+// completion (griddepcontrol.wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), int grid, int smem, cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -277,21 +357,16 @@ mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t col
         const int64_t cap = (int64_t)d->sms * d->occ_tma[dim_m ? 1 : 0];
         const int grid = (int)(work < cap ? work : cap);
         if (dim_m)
-            rearrange_tma<true><<<grid, kThreads, tma_smem_bytes<true>(), stream>>>(map, ends, out, (int64_t)size, s);
+            launch_pdl(rearrange_tma<true>, grid, tma_smem_bytes<true>(), stream, map, ends, out, (int64_t)size, s);
         else
-            rearrange_tma<false><<<grid, kThreads, tma_smem_bytes<false>(), stream>>>(map, ends, out, (int64_t)size, s);
+            launch_pdl(rearrange_tma<false>, grid, tma_smem_bytes<false>(), stream, map, ends, out, (int64_t)size, s);
     } else {
         const int64_t cap = (int64_t)d->sms * d->occ_fallback * 4;
         const int grid = (int)(work < cap ? work : cap);
         const bool word = path == MX_PATH_WORD;
-        if (dim_m && word)
-            rearrange_fallback<true, true><<<grid, kThreads, 0, stream>>>(scales, row_stride, ends, out, (int64_t)size, s);
-        else if (dim_m)
-            rearrange_fallback<true, false><<<grid, kThreads, 0, stream>>>(scales, row_stride, ends, out, (int64_t)size, s);
-        else if (word)
-            rearrange_fallback<false, true><<<grid, kThreads, 0, stream>>>(scales, row_stride, ends, out, (int64_t)size, s);
-        else
-            rearrange_fallback<false, false><<<grid, kThreads, 0, stream>>>(scales, row_stride, ends, out, (int64_t)size, s);
+        auto kernel = dim_m ? (word ? rearrange_fallback<true, true> : rearrange_fallback<true, false>)
+                            : (word ? rearrange_fallback<false, true> : rearrange_fallback<false, false>);
+        launch_pdl(kernel, grid, 0, stream, scales, row_stride, ends, out, (int64_t)size, s);
     }
     return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
