@@ -32,7 +32,7 @@ namespace mx {
 // Error flags written by kernels (read back by mx_device_flags).
 __device__ unsigned int g_mx_flags = 0;
 
-constexpr int kStages = 4;       // input boxes in flight per CTA
+constexpr int kStages = 2;       // input boxes in flight per CTA (3 CTAs per SM)
 constexpr int kOutBuffers = 2;   // output staging blocks per CTA
 constexpr int kOutBytes = kTilesPerChunk * 512;
 
@@ -76,8 +76,22 @@ rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restric
         for (int st = 0; st < kStages; ++st) mbar_init(&full[st], 1);
         fence_mbar_init();
     }
+    // Warm L2 with the boxes this CTA most likely loads first while the
+    // previous kernel drains and before the group scan is known: item i is
+    // placed as if no group were padded.  A prefetch has no observable value,
+    // so it may run before the dependency wait.
+    if (tid == 32) {
+        const int per_band = (s.cols + kChunkCols - 1) / kChunkCols + s.G / 2;
+        for (int n = 0; n < kStages; ++n) {
+            const int i = (int)blockIdx.x + n * (int)gridDim.x;
+            const int y = kDimM ? kTileRows * (i / s.col_chunks) : kTileRows * (i / per_band);
+            const int x = kDimM ? kChunkCols * (i % s.col_chunks)
+                                : min(kChunkCols * (i % per_band), s.cols - 1) & ~15;
+            if (y < s.rows) tma_prefetch_l2(&tmap, x, y);
+        }
+    }
     // Inputs may come from the previous kernel in the stream; outputs may
-    // still be read by it.  Nothing global is touched before this point.
+    // still be read by it.  No global load or store happens before this point.
     grid_dependency_wait();
     if (q == 0) build_group_table<kDimM>(ends, s.G, kDimM ? s.rows : s.cols, s.col_chunks, table);
     __syncthreads();
@@ -166,6 +180,16 @@ rearrange_fallback(const uint8_t *__restrict__ scales, int64_t row_stride, const
     const int j = tid & 31;
     const int q = tid >> 5;
 
+    // L2 prefetch of the rows this CTA most likely handles first (M: item i
+    // is row block i / col_chunks if no group were padded), before the wait.
+    if (kDimM && s.cols <= kChunkCols) {
+        const int64_t y = (int64_t)kTileRows * blockIdx.x;
+        const int64_t span = (int64_t)kTileRows * row_stride;
+        const int64_t off = (int64_t)tid * 128;
+        const int64_t extent = (int64_t)(s.rows - 1) * row_stride + s.cols;   // bytes the view spans
+        if (y < s.rows && off < span && y * row_stride + off < extent)
+            prefetch_l2(scales + y * row_stride + off);
+    }
     grid_dependency_wait();
     if (q == 0) build_group_table<kDimM>(ends, s.G, kDimM ? s.rows : s.cols, s.col_chunks, table);
     __syncthreads();
