@@ -265,6 +265,7 @@ def run_ours(args, rank, world, local):
     import torch
 
     import scale_factor_layout_b200 as mxs
+    from scale_factor_layout_b200 import _binding as B
     from scale_factor_layout_b200 import _build
 
     _build.build()
@@ -345,15 +346,16 @@ def run_ours(args, rank, world, local):
     for c, b, t in zip(cases, per_call, avg):
         gbs = (b["read"] + b["written"]) / t / 1e9
         path = mxs.mx_select_path(c.dim, rot[cases.index(c)][0][1].data_ptr(), c.rows, c.cols, c.cols)
-        calls.append({"case": c.name, "path": {1: "tma", 2: "word", 3: "byte"}.get(path, "?"),
+        calls.append({"case": c.name, "path": B.PATH_NAMES.get(path, "?"),
                       "us": round(t * 1e6, 3), "gbps": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
                       "read_bytes": b["read"], "written_bytes": b["written"], "alloc_bytes": b["alloc"],
                       "gbps_pages_convention": round((b["read"] + b["alloc"]) / t / 1e9, 1)})
     dom = max(range(ncalls), key=lambda i: avg[i])
     dc = calls[dom]
     achieved = dc["read_bytes"] + dc["written_bytes"]
-    roofline = {"bound": "hbm", "kernel": f"rearrange_tma ({dc['case']})" if dc["path"] == "tma"
-                else f"rearrange_fallback ({dc['case']})",
+    kernel_names = {"tma": "rearrange_tma", "flat": "rearrange_flat_tma", "word": "rearrange_fallback",
+                    "byte": "rearrange_fallback"}
+    roofline = {"bound": "hbm", "kernel": f"{kernel_names.get(dc['path'], '?')} ({dc['case']})",
                 "achieved": round(achieved / avg[dom] / 1e9, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / avg[dom] / 1e9 / peak, 4), "peak_source": f"{peak_src} hbm_gbs",
                 "traffic": ncu_traffic(dc["case"]), "algorithmic_bytes": achieved}

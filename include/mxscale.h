@@ -70,11 +70,15 @@ typedef enum {
 
 typedef enum { MX_GROUPS_M = 0, MX_GROUPS_K = 1 } mx_group_dim;
 
-/* Kernel choice.  AUTO takes TMA when `scales` is 16-byte aligned and the
- * row stride is a multiple of 16 bytes; otherwise WORD when both are
- * multiples of 4; otherwise BYTE.  Forcing a path whose rule fails returns
- * MX_ERR_MISALIGNED. */
-typedef enum { MX_PATH_AUTO = 0, MX_PATH_TMA = 1, MX_PATH_WORD = 2, MX_PATH_BYTE = 3 } mx_path;
+/* Kernel choice.  AUTO takes, in order of preference:
+ *   TMA   2-D tensor-map loads: `scales` 16-byte aligned, row stride a multiple of 16;
+ *   FLAT  1-D tensor-map loads of whole row blocks (groups along M only): `scales`
+ *         16-byte aligned, row stride and cols multiples of 4, row stride <= 256;
+ *   WORD  32-bit loads: `scales` and the row stride multiples of 4;
+ *   BYTE  byte loads: anything else.
+ * Forcing a path whose alignment rule fails returns MX_ERR_MISALIGNED; forcing
+ * FLAT for groups along K or a stride above 256 returns MX_ERR_UNSUPPORTED. */
+typedef enum { MX_PATH_AUTO = 0, MX_PATH_TMA = 1, MX_PATH_WORD = 2, MX_PATH_BYTE = 3, MX_PATH_FLAT = 4 } mx_path;
 
 #define MX_MAX_GROUPS 64
 

@@ -17,9 +17,11 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "mxscale.h")
 
 MX_OK, MX_ERR_INVALID_ARG, MX_ERR_MISALIGNED, MX_ERR_UNSUPPORTED, MX_ERR_CUDA = range(5)
 MX_GROUPS_M, MX_GROUPS_K = 0, 1
-MX_PATH_AUTO, MX_PATH_TMA, MX_PATH_WORD, MX_PATH_BYTE = range(4)
+MX_PATH_AUTO, MX_PATH_TMA, MX_PATH_WORD, MX_PATH_BYTE, MX_PATH_FLAT = range(5)
 MX_MAX_GROUPS = 64
-PATHS = {"auto": MX_PATH_AUTO, "tma": MX_PATH_TMA, "word": MX_PATH_WORD, "byte": MX_PATH_BYTE}
+PATHS = {"auto": MX_PATH_AUTO, "tma": MX_PATH_TMA, "word": MX_PATH_WORD, "byte": MX_PATH_BYTE,
+         "flat": MX_PATH_FLAT}
+PATH_NAMES = {v: k for k, v in PATHS.items()}
 
 _lock = threading.Lock()
 _lib = None

@@ -79,6 +79,20 @@ __device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap *map, int x, i
                  ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
 }
 
+// 1-D variants: a box of consecutive elements starting at element x.
+__device__ __forceinline__ void tma_load_1d(void *dst, const CUtensorMap *map, int x, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2}], [%3];"
+        ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_l2_1d(const CUtensorMap *map, int x) {
+    asm volatile("cp.async.bulk.prefetch.tensor.1d.L2.global.tile [%0, {%1}];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x) : "memory");
+}
+
 // Bring the 128-byte line holding p into L2.
 __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));

@@ -163,6 +163,165 @@ rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restric
     if (tid == 0) bulk_wait_all();
 }
 
+// Flat-row TMA kernel (groups along M) for narrow rows whose stride is a
+// multiple of 4 but not of 16 bytes (e.g. 44 columns), where a 2-D tensor map
+// cannot be built.  The scales are viewed as one 1-D array of 32-bit words;
+// an item is a whole 128-row block of a group, which spans
+// delta + rows * row_stride consecutive bytes, loaded as 1 KB boxes from the
+// 16-byte boundary at or below its first byte (boxes past the array's end
+// read zeros).  Rows sit at pitch row_stride in shared memory; with the
+// stride a multiple of 4 every row starts on a word, and the transpose reads
+// 32-bit words.  Pipeline, staging and bulk stores follow rearrange_tma.
+constexpr int kFlatBoxWords = 256;
+constexpr int kFlatBoxBytes = kFlatBoxWords * 4;
+constexpr int kFlatStages = 4;
+constexpr int kFlatMaxStride = 256;
+
+struct FlatShape {
+    int32_t row_stride;     // bytes, a multiple of 4
+    int32_t stage_bytes;    // boxes per stage * 1 KB
+    int32_t staging_bytes;  // tiles per row block * 512, rounded to 1 KB
+};
+
+__global__ void __launch_bounds__(kThreads)
+rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restrict__ ends,
+                   uint8_t *__restrict__ out, int64_t out_size, Shape s, FlatShape f) {
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t *stages = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(dyn_smem) + 127) & ~uintptr_t(127));
+    uint8_t *staging = stages + kFlatStages * f.stage_bytes;
+    __shared__ GroupTable table;
+    __shared__ __align__(8) uint64_t full[kFlatStages];
+    __shared__ Item items[kFlatStages];
+
+    const int tid = threadIdx.x;
+    const int j = tid & 31;
+    const int q = tid >> 5;
+    const int L = f.row_stride;
+    const int ntiles = s.padded_cols / 4;     // every item covers all columns
+    const int nquads = (ntiles + 3) / 4;
+
+    if (tid == 0) {
+        tma_prefetch_desc(&tmap);
+#pragma unroll
+        for (int st = 0; st < kFlatStages; ++st) mbar_init(&full[st], 1);
+        fence_mbar_init();
+    }
+    // L2 prefetch of the row blocks this CTA most likely takes first (row
+    // block i if no group were padded); no observable value, so before the wait.
+    if (tid == 32) {
+        for (int n = 0; n < kFlatStages; ++n) {
+            const int64_t y = (int64_t)kTileRows * ((int)blockIdx.x + n * (int)gridDim.x);
+            if (y >= s.rows) break;
+            const int64_t w0 = ((y * L) >> 4) << 2;
+            for (int b = 0; b * kFlatBoxBytes < kTileRows * L; ++b)
+                tma_prefetch_l2_1d(&tmap, (int)(w0 + b * kFlatBoxWords));
+        }
+    }
+    grid_dependency_wait();
+    if (q == 0) build_group_table<true>(ends, s.G, s.rows, 1, table);
+    __syncthreads();
+    grid_launch_dependents();
+
+    const int total = table.istart[kMaxGroups];
+    const int bid = blockIdx.x;
+    const int n_my = bid < total ? (total - 1 - bid) / (int)gridDim.x + 1 : 0;
+
+    auto issue = [&](int n, int st) {
+        const int i = bid + n * (int)gridDim.x;
+        const int g = find_group(table, s.G, i);
+        const int rb = i - table.istart[g];
+        Item it;
+        it.y = table.begin[g] + rb * kTileRows;
+        it.rows_valid = min(kTileRows, table.size[g] - rb * kTileRows);
+        it.cols_valid = s.cols;
+        it.ntiles = ntiles;
+        it.out_off = ((int64_t)table.pstart[g] + (int64_t)rb * kTileRows) * s.padded_cols;
+        const int64_t byte0 = (int64_t)it.y * L;
+        const int64_t word0 = (byte0 >> 4) << 2;
+        it.delta = (int)(byte0 - word0 * 4);
+        const int nbox = (it.delta + it.rows_valid * L + kFlatBoxBytes - 1) / kFlatBoxBytes;
+        it.x = (int)word0;
+        items[st] = it;
+        mbar_arrive_expect_tx(&full[st], (uint32_t)nbox * kFlatBoxBytes);
+        for (int b = 0; b < nbox; ++b)
+            tma_load_1d(stages + st * f.stage_bytes + b * kFlatBoxBytes, &tmap, it.x + b * kFlatBoxWords, &full[st]);
+    };
+
+    if (tid == 0)
+        for (int st = 0; st < kFlatStages && st < n_my; ++st) issue(st, st);
+
+    int64_t prev_off = 0;
+    uint32_t prev_bytes = 0;
+    for (int n = 0; n < n_my; ++n) {
+        const int st = n % kFlatStages;
+        const uint32_t parity = (uint32_t)(n / kFlatStages) & 1u;
+        const bool ok = mbar_wait_bounded(&full[st], parity);
+        Item it;
+        uint32_t wv[2][4][4];   // [quad pass][row a][word t]
+        if (ok) {
+            it = items[st];
+            const uint8_t *stage = stages + st * f.stage_bytes + it.delta;
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const int qq = q + 8 * p;
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    const uint32_t *row = reinterpret_cast<const uint32_t *>(stage + (j + 32 * a) * L) + 4 * qq;
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) wv[p][a][t] = (qq < nquads) ? row[t] : 0u;
+                }
+            }
+        }
+        if (tid == 0) bulk_wait_read<0>();
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_mx_flags, kFlagWaitTimeout);
+                for (int m = n; m < n_my && m < n + kFlatStages; ++m)
+                    mbar_wait_bounded(&full[m % kFlatStages], (uint32_t)(m / kFlatStages) & 1u);
+            }
+            return;
+        }
+        if (tid == 0) {
+            if (n > 0) {
+                bulk_store_s2g(out + prev_off, staging + ((n - 1) & 1) * f.staging_bytes, prev_bytes);
+                bulk_commit();
+            }
+            prev_off = it.out_off;
+            prev_bytes = (uint32_t)it.ntiles * 512u;
+            if (n + kFlatStages < n_my) issue(n + kFlatStages, st);
+        }
+        uint8_t *stg = staging + (n & 1) * f.staging_bytes;
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const int qq = q + 8 * p;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int tile = 4 * qq + t;
+                if (qq < nquads && tile < ntiles) {
+                    // columns 4*tile.. are all real (cols is a multiple of 4 here)
+                    uint4 o;
+                    o.x = (j < it.rows_valid) ? wv[p][0][t] : 0u;
+                    o.y = (j + 32 < it.rows_valid) ? wv[p][1][t] : 0u;
+                    o.z = (j + 64 < it.rows_valid) ? wv[p][2][t] : 0u;
+                    o.w = (j + 96 < it.rows_valid) ? wv[p][3][t] : 0u;
+                    *reinterpret_cast<uint4 *>(stg + tile * 512 + 16 * j) = o;
+                }
+            }
+        }
+        fence_proxy_async_smem();
+    }
+    if (n_my > 0) {
+        __syncthreads();
+        if (tid == 0) {
+            bulk_store_s2g(out + prev_off, staging + ((n_my - 1) & 1) * f.staging_bytes, prev_bytes);
+            bulk_commit();
+        }
+    }
+    zero_tail(out, (int64_t)table.pstart[kMaxGroups] * s.padded_cols, out_size);
+    if (tid == 0) bulk_wait_all();
+}
+
 // Fallback for any stride and alignment.  One work item per loop trip: every
 // thread first issues all of its loads for the item (up to kMaxWordsPerThread
 // 32-bit words, or their bytes), then parks them in shared memory; the
@@ -253,6 +412,18 @@ struct DeviceInfo {
     int occ_fallback = 0;
 };
 
+// Shared memory of the flat-row kernel for a given row stride and column count.
+FlatShape flat_shape(int64_t row_stride, int64_t padded_cols) {
+    FlatShape f;
+    f.row_stride = (int32_t)row_stride;
+    const int64_t span = 16 + kTileRows * row_stride + 256;   // delta, rows, last partial quad
+    f.stage_bytes = (int32_t)((span + kFlatBoxBytes - 1) / kFlatBoxBytes * kFlatBoxBytes);
+    f.staging_bytes = (int32_t)(((padded_cols / 4) * 512 + 1023) / 1024 * 1024);
+    return f;
+}
+
+int flat_smem_bytes(const FlatShape &f) { return kFlatStages * f.stage_bytes + 2 * f.staging_bytes + 128; }
+
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -276,7 +447,10 @@ mx_status device_info(const DeviceInfo **out) {
     DeviceInfo &d = g_dev[dev];
     if (!d.ready) {
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MX_ERR_CUDA;
-        if (cudaFuncSetAttribute(rearrange_tma<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        const int flat_max = flat_smem_bytes(flat_shape(kFlatMaxStride, kFlatMaxStride));
+        if (cudaFuncSetAttribute(rearrange_flat_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, flat_max) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(rearrange_tma<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tma_smem_bytes<true>()) != cudaSuccess ||
             cudaFuncSetAttribute(rearrange_tma<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tma_smem_bytes<false>()) != cudaSuccess)
@@ -325,10 +499,27 @@ bool word_eligible(const void *scales, int64_t row_stride) {
     return (reinterpret_cast<uintptr_t>(scales) & 3u) == 0 && (row_stride & 3) == 0;
 }
 
+bool flat_aligned(const void *scales, int64_t cols, int64_t row_stride) {
+    return (reinterpret_cast<uintptr_t>(scales) & 15u) == 0 && (row_stride & 3) == 0 && (cols & 3) == 0;
+}
+
+bool flat_eligible(mx_group_dim dim, const void *scales, int64_t rows, int64_t cols, int64_t row_stride) {
+    return dim == MX_GROUPS_M && rows >= 1 && cols >= 1 && row_stride <= kFlatMaxStride &&
+           flat_aligned(scales, cols, row_stride) && ((rows - 1) * row_stride + cols) / 4 < INT_MAX - (1 << 16);
+}
+
+mx_path auto_path(mx_group_dim dim, const void *scales, int64_t rows, int64_t cols, int64_t row_stride) {
+    if (rows == 0 || cols == 0) return MX_PATH_WORD;   // nothing to load
+    if (tma_eligible(scales, rows, cols, row_stride)) return MX_PATH_TMA;
+    if (flat_eligible(dim, scales, rows, cols, row_stride)) return MX_PATH_FLAT;
+    if (word_eligible(scales, row_stride)) return MX_PATH_WORD;
+    return MX_PATH_BYTE;
+}
+
 mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t cols, int64_t row_stride,
               const int32_t *ends, int32_t G, uint8_t *out, mx_path path, cudaStream_t stream) {
     if (dim != MX_GROUPS_M && dim != MX_GROUPS_K) return MX_ERR_INVALID_ARG;
-    if (path < MX_PATH_AUTO || path > MX_PATH_BYTE) return MX_ERR_INVALID_ARG;
+    if (path < MX_PATH_AUTO || path > MX_PATH_FLAT) return MX_ERR_INVALID_ARG;
     if (G < 1 || G > MX_MAX_GROUPS) return MX_ERR_INVALID_ARG;
     if (rows < 0 || cols < 0 || rows > kMaxExtent || cols > kMaxExtent) return MX_ERR_INVALID_ARG;
     if (row_stride < cols) return MX_ERR_INVALID_ARG;
@@ -353,12 +544,11 @@ mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t col
     if (bound > INT_MAX) return MX_ERR_UNSUPPORTED;
 
     const bool degenerate = rows == 0 || cols == 0;
-    if (path == MX_PATH_AUTO)
-        path = tma_eligible(scales, rows, cols, row_stride) ? MX_PATH_TMA
-               : word_eligible(scales, row_stride)          ? MX_PATH_WORD
-                                                            : MX_PATH_BYTE;
+    if (path == MX_PATH_AUTO) path = auto_path(dim, scales, rows, cols, row_stride);
     if (degenerate) path = MX_PATH_WORD;  // nothing to load: only the zero fill runs
     if (path == MX_PATH_TMA && !tma_eligible(scales, rows, cols, row_stride)) return MX_ERR_MISALIGNED;
+    if (path == MX_PATH_FLAT && (!dim_m || row_stride > kFlatMaxStride)) return MX_ERR_UNSUPPORTED;
+    if (path == MX_PATH_FLAT && !flat_eligible(dim, scales, rows, cols, row_stride)) return MX_ERR_MISALIGNED;
     if (path == MX_PATH_WORD && !degenerate && !word_eligible(scales, row_stride)) return MX_ERR_MISALIGNED;
 
     const DeviceInfo *d = nullptr;
@@ -384,6 +574,27 @@ mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t col
             launch_pdl(rearrange_tma<true>, grid, tma_smem_bytes<true>(), stream, map, ends, out, (int64_t)size, s);
         else
             launch_pdl(rearrange_tma<false>, grid, tma_smem_bytes<false>(), stream, map, ends, out, (int64_t)size, s);
+    } else if (path == MX_PATH_FLAT) {
+        auto encode = encode_fn();
+        if (encode == nullptr) return MX_ERR_CUDA;
+        CUtensorMap map;
+        cuuint64_t gdim[1] = {(cuuint64_t)(((rows - 1) * row_stride + cols) / 4)};
+        cuuint64_t gstride[1] = {0};
+        cuuint32_t box[1] = {(cuuint32_t)kFlatBoxWords};
+        cuuint32_t estride[1] = {1};
+        CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 1, const_cast<uint8_t *>(scales), gdim, gstride,
+                            box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return MX_ERR_CUDA;
+        const FlatShape f = flat_shape(row_stride, s.padded_cols);
+        const int smem = flat_smem_bytes(f);
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rearrange_flat_tma, kThreads, smem) != cudaSuccess ||
+            occ < 1)
+            return MX_ERR_CUDA;
+        const int64_t cap = (int64_t)d->sms * occ;
+        const int grid = (int)(work < cap ? work : cap);
+        launch_pdl(rearrange_flat_tma, grid, smem, stream, map, ends, out, (int64_t)size, s, f);
     } else {
         const int64_t cap = (int64_t)d->sms * d->occ_fallback * 4;
         const int grid = (int)(work < cap ? work : cap);
@@ -429,10 +640,7 @@ mx_status mx_rearrange_ex(mx_group_dim dim, const uint8_t *scales, int64_t rows,
 }
 
 mx_path mx_select_path(mx_group_dim dim, const void *scales, int64_t rows, int64_t cols, int64_t row_stride) {
-    (void)dim;
-    if (mx::tma_eligible(scales, rows, cols, row_stride)) return MX_PATH_TMA;
-    if (mx::word_eligible(scales, row_stride) || rows == 0 || cols == 0) return MX_PATH_WORD;
-    return MX_PATH_BYTE;
+    return mx::auto_path(dim, scales, rows, cols, row_stride);
 }
 
 const char *mx_status_string(mx_status status) {

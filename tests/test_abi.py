@@ -31,7 +31,10 @@ def test_sizes_match_oracle(mxlib, orc):
 
 def test_path_selection(mxlib):
     assert B.mx_select_path(M, 0x1000, 100, 224, 224) == B.MX_PATH_TMA
-    assert B.mx_select_path(M, 0x1000, 100, 44, 44) == B.MX_PATH_WORD
+    assert B.mx_select_path(M, 0x1000, 100, 44, 44) == B.MX_PATH_FLAT      # narrow rows, stride % 16 != 0
+    assert B.mx_select_path(M, 0x1000, 100, 44, 300) == B.MX_PATH_WORD     # stride above the flat limit
+    assert B.mx_select_path(M, 0x1000, 100, 43, 44) == B.MX_PATH_WORD      # cols not a multiple of 4
+    assert B.mx_select_path(K, 0x1000, 100, 44, 44) == B.MX_PATH_WORD      # flat is M-groups only
     assert B.mx_select_path(M, 0x1004, 100, 48, 48) == B.MX_PATH_WORD      # base not 16-aligned
     assert B.mx_select_path(K, 0x1000, 100, 45, 45) == B.MX_PATH_BYTE      # odd stride
     assert B.mx_select_path(K, 0x1001, 100, 48, 48) == B.MX_PATH_BYTE      # odd base
@@ -61,6 +64,11 @@ def _call(dim=M, scales=0x1000, rows=256, cols=64, stride=64, ends=0x2000, G=2, 
     (dict(stride=66, path=B.MX_PATH_WORD), B.MX_ERR_MISALIGNED),
     (dict(scales=0x1002, path=B.MX_PATH_WORD), B.MX_ERR_MISALIGNED),
     (dict(dim=K, rows=0), B.MX_OK),          # empty allocation: nothing to do, no launch
+    (dict(dim=K, cols=44, stride=44, path=B.MX_PATH_FLAT), B.MX_ERR_UNSUPPORTED),
+    (dict(cols=44, stride=300, path=B.MX_PATH_FLAT), B.MX_ERR_UNSUPPORTED),
+    (dict(cols=44, stride=44, scales=0x1004, path=B.MX_PATH_FLAT), B.MX_ERR_MISALIGNED),
+    (dict(cols=43, stride=44, path=B.MX_PATH_FLAT), B.MX_ERR_MISALIGNED),
+    (dict(path=5), B.MX_ERR_INVALID_ARG),
 ])
 def test_host_validation(mxlib, kwargs, status):
     assert _call(**kwargs) == status

@@ -38,10 +38,15 @@ def test_workloads_auto(mxlib, orc, cases, name):
     _check(cases[name], orc)
 
 
+def flat_ok(c, ptr):
+    return (c.dim == synth.DIM_M and ptr % 16 == 0 and c.row_stride % 4 == 0 and c.cols % 4 == 0
+            and c.row_stride <= 256 and c.rows >= 1 and c.cols >= 1)
+
+
 @pytest.mark.parametrize("name,path", [
-    ("m_tiny", "word"), ("m_tiny", "byte"),
-    ("m_skinny", "word"), ("m_skinny", "byte"),
-    ("m_wide", "tma"), ("m_wide", "word"), ("m_wide", "byte"),
+    ("m_tiny", "flat"), ("m_tiny", "word"), ("m_tiny", "byte"),
+    ("m_skinny", "flat"), ("m_skinny", "word"), ("m_skinny", "byte"),
+    ("m_wide", "tma"), ("m_wide", "flat"), ("m_wide", "word"), ("m_wide", "byte"),
     ("k_groups", "tma"), ("k_groups", "word"), ("k_groups", "byte"),
 ])
 def test_workloads_forced_path(mxlib, orc, cases, name, path):
@@ -49,7 +54,7 @@ def test_workloads_forced_path(mxlib, orc, cases, name, path):
 
 
 def test_auto_dispatch_choices(mxlib, cases):
-    for name, want in (("m_tiny", B.MX_PATH_WORD), ("m_skinny", B.MX_PATH_WORD),
+    for name, want in (("m_tiny", B.MX_PATH_FLAT), ("m_skinny", B.MX_PATH_FLAT),
                        ("m_wide", B.MX_PATH_TMA), ("k_groups", B.MX_PATH_TMA)):
         c = cases[name]
         dc = DeviceCase(c)
@@ -65,6 +70,8 @@ def test_k_sweep(mxlib, orc, i_rows):
 @pytest.mark.parametrize("name,pad,path", [
     ("m_wide", 32, "auto"), ("k_groups", 32, "auto"),   # stride still a multiple of 16: TMA with gaps
     ("m_wide", 4, "auto"), ("k_groups", 4, "auto"),     # word path
+    ("m_skinny", 4, "auto"), ("m_skinny", 20, "flat"),  # flat path with gaps between rows
+    ("m_tiny", 8, "flat"),
     ("m_skinny", 5, "auto"), ("k_groups", 5, "auto"),   # byte path
     ("m_tiny", 19, "auto"),
 ])
@@ -74,7 +81,7 @@ def test_strided(mxlib, orc, cases, name, pad, path):
 
 @pytest.mark.parametrize("misalign", [1, 2, 4, 8, 12])
 def test_misaligned_base(mxlib, orc, misalign):
-    for c in (synth.m_tiny(), synth.k_sweep_point(1, 3)):
+    for c in (synth.m_tiny(), synth.k_sweep_point(1, 3), synth.m_wide()):
         _check(c, orc, misalign=misalign)
 
 
@@ -92,8 +99,11 @@ def test_random_small(mxlib, orc, chunk):
         c = synth.random_small(seed)
         paths = ["auto", "byte"]
         dc = DeviceCase(c)
-        if B.mx_select_path(c.dim, dc.ptr, c.rows, c.cols, c.row_stride) == B.MX_PATH_TMA:
+        auto = B.mx_select_path(c.dim, dc.ptr, c.rows, c.cols, c.row_stride)
+        if auto in (B.MX_PATH_TMA, B.MX_PATH_FLAT):
             paths.append("word")
+        if auto == B.MX_PATH_TMA and flat_ok(c, dc.ptr):
+            paths.append("flat")
         for p in paths:
             _check(c, orc, p)
 
@@ -115,7 +125,7 @@ def test_max_groups_and_empty(mxlib, orc):
                 sizes = np.ones(64, np.int64); sizes[-1] = total - 63
             s = synth.uniform_scales(rng, rows, cols, 100, 140)
             c = synth.Case(f"g64_{pattern}", dim, s, synth.ends_from_sizes(sizes), 0)
-            for p in ("auto", "word"):
+            for p in ("auto", "word") + (("flat",) if flat_ok(c, 0) else ()):
                 _check(c, orc, p)
 
 
