@@ -3,7 +3,7 @@
 
 One step = one pass of the hot path over one batch of synthetic scales: the
 three production shapes of the pytorch/ao pages, each one C-ABI call:
-  * M-groups (131072, 44), G=8  -- the DSV3-16b shape of #3708 (fallback path)
+  * M-groups (131072, 44), G=8  -- the DSV3-16b shape of #3708 (flat-row TMA path)
   * M-groups (131072, 224), G=8 -- data K = 7168 (TMA path)
   * K-groups (7168, 4096), G=8  -- data K = 131072 tokens (TMA path)
 Metric: GB/s = (bytes of real scales read + exact padded bytes written) / time,
@@ -44,8 +44,8 @@ WORKLOADS = {
     "k_groups": ["k_groups"],
 }
 WORKLOAD_DESC = {
-    "moe_step": "M-groups 131072x44 G=8 (fallback) + M-groups 131072x224 G=8 (TMA) + K-groups 7168x4096 G=8 (TMA)",
-    "m_skinny": "M-groups 131072x44 G=8, stride 44 B (fallback)",
+    "moe_step": "M-groups 131072x44 G=8 (flat-row TMA) + M-groups 131072x224 G=8 (TMA) + K-groups 7168x4096 G=8 (TMA)",
+    "m_skinny": "M-groups 131072x44 G=8, stride 44 B (flat-row TMA)",
     "m_wide": "M-groups 131072x224 G=8 (TMA)",
     "k_groups": "K-groups 7168x4096 G=8 (TMA)",
 }
@@ -82,7 +82,32 @@ def algorithmic_bytes(case) -> dict:
 def make_cases(workload: str):
     from scale_factor_layout_b200 import synth
 
+    if workload.startswith("k_sweep_"):
+        m, total_k = (int(v) for v in workload[len("k_sweep_"):].split("x"))
+        return [synth.k_sweep_point(synth.SWEEP_ROWS.index(m), synth.SWEEP_TOTAL_K.index(total_k))]
     return [synth.NAMED[name]() for name in WORKLOADS[workload]]
+
+
+def workload_desc(workload: str) -> str:
+    if workload.startswith("k_sweep_"):
+        m, total_k = (int(v) for v in workload[len("k_sweep_"):].split("x"))
+        return f"K-groups sweep point M={m} TotalK={total_k}: scales {m}x{total_k // 32}, G=8 (TMA)"
+    return WORKLOAD_DESC[workload]
+
+
+def workload_arg(value: str) -> str:
+    from scale_factor_layout_b200 import synth
+
+    if value in WORKLOADS:
+        return value
+    if value.startswith("k_sweep_"):
+        try:
+            m, total_k = (int(v) for v in value[len("k_sweep_"):].split("x"))
+            if m in synth.SWEEP_ROWS and total_k in synth.SWEEP_TOTAL_K:
+                return value
+        except ValueError:
+            pass
+    raise argparse.ArgumentTypeError(f"unknown workload {value!r}: one of {sorted(WORKLOADS)} or k_sweep_<M>x<TotalK>")
 
 
 # ------------------------------------------------------------------ environment
@@ -366,7 +391,7 @@ def run_ours(args, rank, world, local):
         "warmup": args.warmup, "ms_per_step": round(seconds_max / args.steps * 1e3, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
         "data": "synthetic (seeded uniform E8M0 bytes, seeded group splits)",
-        "config": {"workload": args.workload, "description": WORKLOAD_DESC[args.workload],
+        "config": {"workload": args.workload, "description": workload_desc(args.workload),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "bytes_per_step": step_bytes, "bytes_per_step_pages_convention": step_bytes_pages,
                    "l2": "inputs/outputs rotate per call over " + ", ".join(str(len(r)) for r in rot)
@@ -504,7 +529,7 @@ def run_reference(args, rank, world):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(seconds / args.steps * 1e3, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
            "data": "synthetic (seeded uniform E8M0 bytes, seeded group splits)",
-           "config": {"workload": args.workload, "description": WORKLOAD_DESC[args.workload],
+           "config": {"workload": args.workload, "description": workload_desc(args.workload),
                       "parallelism": "single host thread"},
            "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
                             "sample": f"{desc}, single thread, gcc -O2, {cpu_model()}"},
@@ -518,7 +543,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="moe_step")
+    ap.add_argument("--workload", type=workload_arg, default="moe_step",
+                    help=f"one of {sorted(WORKLOADS)} or k_sweep_<M>x<TotalK> (a point of the K-groups sweep)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -128,6 +128,13 @@ const char *mx_status_string(mx_status status);
  * the flags after reading. */
 mx_status mx_device_flags(uint32_t *flags, int clear);
 
+/* Failure-detection self-test: launches one CTA that waits, with the same
+ * bounded mbarrier wait the pipelines use, on a barrier nothing arrives at.
+ * The wait gives up after `limit_cycles` SM clocks (1 .. 2^32) and sets bit 0
+ * of the device flags; read them with mx_device_flags.  The kernel returns
+ * normally and the context stays usable.  Asynchronous on `stream`. */
+mx_status mx_selftest_bounded_wait(int64_t limit_cycles, cudaStream_t stream);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int mx_version(void);
 

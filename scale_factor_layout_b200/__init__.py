@@ -12,7 +12,8 @@ from __future__ import annotations
 from ._binding import (  # noqa: F401
     MX_GROUPS_K, MX_GROUPS_M, MX_MAX_GROUPS, MX_OK, MX_PATH_AUTO, MX_PATH_BYTE, MX_PATH_TMA,
     MX_PATH_WORD, PATHS, MxError, declared_symbols, lib, mx_device_flags, mx_rearrange_ex,
-    mx_rearrange_k_groups, mx_rearrange_m_groups, mx_rearranged_size, mx_select_path, mx_version,
+    mx_rearrange_k_groups, mx_rearrange_m_groups, mx_rearranged_size, mx_select_path,
+    mx_selftest_bounded_wait, mx_version,
     status_string,
 )
 

@@ -36,6 +36,7 @@ _SIGNATURES = {
     "mx_select_path": (ctypes.c_int, [ctypes.c_int, _P, _I64, _I64, _I64]),
     "mx_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mx_device_flags": (ctypes.c_int, [_U32P, ctypes.c_int]),
+    "mx_selftest_bounded_wait": (ctypes.c_int, [_I64, _P]),
     "mx_version": (ctypes.c_int, []),
 }
 
@@ -105,6 +106,10 @@ def mx_device_flags(clear: bool = False) -> int:
     if st != MX_OK:
         raise MxError("mx_device_flags", st)
     return int(v.value)
+
+
+def mx_selftest_bounded_wait(limit_cycles: int, stream: int = 0) -> int:
+    return lib().mx_selftest_bounded_wait(limit_cycles, stream)
 
 
 def mx_version() -> int:

@@ -401,6 +401,18 @@ rearrange_fallback(const uint8_t *__restrict__ scales, int64_t row_stride, const
     zero_tail(out, covered_bytes<kDimM>(table, s), out_size);
 }
 
+// Self-test of the bounded pipeline wait: one thread waits on an mbarrier
+// that nothing arrives at; the wait gives up after `limit` clocks and raises
+// the timeout flag, exactly as a stalled load would in the kernels above.
+__global__ void bounded_wait_selftest(long long limit) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        if (!mbar_wait_bounded(&bar, 0, limit)) atomicOr(&g_mx_flags, kFlagWaitTimeout);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 constexpr int64_t kMaxExtent = (1ll << 31) - (1ll << 14);
 constexpr int kMaxDevices = 128;
@@ -664,6 +676,12 @@ mx_status mx_device_flags(uint32_t *flags, int clear) {
         if (cudaMemcpyToSymbol(mx::g_mx_flags, &zero, sizeof(zero)) != cudaSuccess) return MX_ERR_CUDA;
     }
     return MX_OK;
+}
+
+mx_status mx_selftest_bounded_wait(int64_t limit_cycles, cudaStream_t stream) {
+    if (limit_cycles < 1 || limit_cycles > (1ll << 32)) return MX_ERR_INVALID_ARG;
+    mx::bounded_wait_selftest<<<1, 32, 0, stream>>>((long long)limit_cycles);
+    return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 
 int mx_version(void) { return 100; }
