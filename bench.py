@@ -254,8 +254,10 @@ def aggregate_value(bytes_per_step: int, steps: int, n_gpus: int, seconds: float
 
 
 # ------------------------------------------------------------------ GPU arm
-def device_copies(case, n, device):
-    """n independent device copies of a case's inputs, each with its own output."""
+def device_copies(case, n, device, op="rearrange"):
+    """n independent device copies of a case's inputs, each with its own output.
+    For the inverse, the input is the blocked layout (made once here by the
+    forward call) and the output a row-major (rows, cols) buffer."""
     import torch
 
     import scale_factor_layout_b200 as mxs
@@ -265,8 +267,13 @@ def device_copies(case, n, device):
     host_e = torch.from_numpy(np.ascontiguousarray(case.ends, dtype=np.int32))
     size = mxs.mx_rearranged_size(case.dim, case.rows, case.cols, case.num_groups)
     for _ in range(n):
-        out.append((case, host_s.to(device), host_e.to(device),
-                    torch.empty(size, dtype=torch.uint8, device=device)))
+        s, e = host_s.to(device), host_e.to(device)
+        if op == "inverse":
+            blocked = mxs.rearrange(case.dim, s, e)
+            out.append((case, blocked, e, torch.empty((case.rows, case.cols), dtype=torch.uint8, device=device)))
+            del s
+        else:
+            out.append((case, s, e, torch.empty(size, dtype=torch.uint8, device=device)))
     return out
 
 
@@ -276,12 +283,16 @@ def rotation_count(case) -> int:
     return max(2, math.ceil(4 * L2_BYTES / (b["read"] + b["alloc"])))
 
 
-def launch(item, stream_handle):
+def launch(item, stream_handle, op="rearrange"):
     from scale_factor_layout_b200 import _binding as B
 
     c, s, e, o = item
-    st = B.mx_rearrange_ex(c.dim, s.data_ptr(), c.rows, c.cols, c.cols, e.data_ptr(), c.num_groups,
-                           o.data_ptr(), B.MX_PATH_AUTO, stream_handle)
+    if op == "inverse":
+        fn = B.mx_unrearrange_m_groups if c.dim == 0 else B.mx_unrearrange_k_groups
+        st = fn(s.data_ptr(), c.rows, c.cols, e.data_ptr(), c.num_groups, o.data_ptr(), c.cols, stream_handle)
+    else:
+        st = B.mx_rearrange_ex(c.dim, s.data_ptr(), c.rows, c.cols, c.cols, e.data_ptr(), c.num_groups,
+                               o.data_ptr(), B.MX_PATH_AUTO, stream_handle)
     if st != B.MX_OK:
         raise RuntimeError(f"{c.name}: {B.status_string(st)}")
 
@@ -302,7 +313,7 @@ def run_ours(args, rank, world, local):
     step_bytes = sum(b["read"] + b["written"] for b in per_call)
     step_bytes_pages = sum(b["read"] + b["alloc"] for b in per_call)
 
-    rot = [device_copies(c, rotation_count(c), device) for c in cases]
+    rot = [device_copies(c, rotation_count(c), device, args.op) for c in cases]
     rot_bytes = sum(len(r) * (algorithmic_bytes(c)["read"] + algorithmic_bytes(c)["alloc"])
                     for c, r in zip(cases, rot))
     stream = torch.cuda.Stream(device)
@@ -315,7 +326,7 @@ def run_ours(args, rank, world, local):
     with torch.cuda.stream(stream):
         for k in range(3):  # first calls set kernel attributes (outside capture) and warm caches
             for it in step_items(k):
-                launch(it, h)
+                launch(it, h, args.op)
     torch.cuda.synchronize()
 
     def capture(launches):
@@ -324,7 +335,7 @@ def run_ours(args, rank, world, local):
         with torch.cuda.stream(stream):
             with torch.cuda.graph(g, stream=stream):
                 for it in launches:
-                    launch(it, h)
+                    launch(it, h, args.op)
         return g
 
     def steps_of(k0, n):
@@ -380,18 +391,23 @@ def run_ours(args, rank, world, local):
     achieved = dc["read_bytes"] + dc["written_bytes"]
     kernel_names = {"tma": "rearrange_tma", "flat": "rearrange_flat_tma", "word": "rearrange_fallback",
                     "byte": "rearrange_fallback"}
-    roofline = {"bound": "hbm", "kernel": f"{kernel_names.get(dc['path'], '?')} ({dc['case']})",
+    kname = "unrearrange_kernel" if args.op == "inverse" else kernel_names.get(dc["path"], "?")
+    roofline = {"bound": "hbm", "kernel": f"{kname} ({dc['case']})",
                 "achieved": round(achieved / avg[dom] / 1e9, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / avg[dom] / 1e9 / peak, 4), "peak_source": f"{peak_src} hbm_gbs",
-                "traffic": ncu_traffic(dc["case"]), "algorithmic_bytes": achieved}
+                "traffic": ncu_traffic(dc["case"]) if args.op == "rearrange" else None,
+                "algorithmic_bytes": achieved}
 
-    e2e = run_e2e(args, cases, device, world, dist) if not args.no_e2e else None
+    if args.op == "inverse":
+        for cl in calls:
+            cl["path"] = "inverse"
+    e2e = run_e2e(args, cases, device, world, dist) if not args.no_e2e and args.op == "rearrange" else None
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(seconds_max / args.steps * 1e3, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
         "data": "synthetic (seeded uniform E8M0 bytes, seeded group splits)",
-        "config": {"workload": args.workload, "description": workload_desc(args.workload),
+        "config": {"workload": args.workload, "op": args.op, "description": workload_desc(args.workload),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "bytes_per_step": step_bytes, "bytes_per_step_pages_convention": step_bytes_pages,
                    "l2": "inputs/outputs rotate per call over " + ", ".join(str(len(r)) for r in rot)
@@ -506,22 +522,30 @@ def run_reference(args, rank, world):
 
     oracle.load()
     cases = make_cases(args.workload)
+
+    def runner(sample):
+        """One step's oracle work: the rearrange, or for --op inverse the
+        oracle's inverse of its own blocked output (made once, outside the timing)."""
+        if args.op == "inverse":
+            blocked = [oracle.rearrange(c.dim, c.scales, c.ends) for c in sample]
+            return lambda: [oracle.inverse(c.dim, b, c.rows, c.cols, c.ends) for c, b in zip(sample, blocked)]
+        return lambda: [oracle.rearrange(c.dim, c.scales, c.ends) for c in sample]
+
+    full = runner(cases)
     t0 = time.perf_counter()
-    for c in cases:
-        oracle.rearrange(c.dim, c.scales, c.ends)
+    full()
     full_step = time.perf_counter() - t0
     budget = 120.0
     fraction = min(1.0, budget / max(1e-9, full_step * (args.steps + args.warmup)))
     sample = cases if fraction >= 1.0 else sample_cases(cases, fraction)
     per = [algorithmic_bytes(c) for c in sample]
     step_bytes = sum(b["read"] + b["written"] for b in per)
+    work = runner(sample)
     for _ in range(args.warmup):
-        for c in sample:
-            oracle.rearrange(c.dim, c.scales, c.ends)
+        work()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        for c in sample:
-            oracle.rearrange(c.dim, c.scales, c.ends)
+        work()
     seconds = time.perf_counter() - t0
     value = step_bytes * args.steps / seconds / 1e9
     desc = "full workload" if fraction >= 1.0 else f"leading {fraction:.3f} of each case's rows"
@@ -529,7 +553,7 @@ def run_reference(args, rank, world):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(seconds / args.steps * 1e3, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
            "data": "synthetic (seeded uniform E8M0 bytes, seeded group splits)",
-           "config": {"workload": args.workload, "description": workload_desc(args.workload),
+           "config": {"workload": args.workload, "op": args.op, "description": workload_desc(args.workload),
                       "parallelism": "single host thread"},
            "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
                             "sample": f"{desc}, single thread, gcc -O2, {cpu_model()}"},
@@ -545,6 +569,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=workload_arg, default="moe_step",
                     help=f"one of {sorted(WORKLOADS)} or k_sweep_<M>x<TotalK> (a point of the K-groups sweep)")
+    ap.add_argument("--op", choices=["rearrange", "inverse"], default="rearrange",
+                    help="rearrange (row-major -> blocked, the hot path) or its inverse")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")

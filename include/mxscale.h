@@ -116,6 +116,35 @@ mx_status mx_rearrange_ex(mx_group_dim dim, const uint8_t *scales, int64_t rows,
                           int64_t row_stride, const int32_t *group_end_offsets, int32_t num_groups,
                           uint8_t *out, mx_path path, cudaStream_t stream);
 
+/* Inverse of mx_rearrange_m_groups: read a blocked buffer (16-byte aligned, laid
+ * out as mx_rearrange_m_groups writes it for the same rows, cols and group
+ * ends) and write the row-major scales: element (i, j) at
+ * scales[i * row_stride + j], any alignment.  Elements that no group covers
+ * (rows at or past the last clamped end) are written as 0; bytes between
+ * cols and row_stride are not touched.  Padding bytes of `blocked` are not
+ * read.  Same limits, clamping and stream rules as the forward call; the
+ * blocked buffer must not overlap `scales`.  (The other side of the layout
+ * the pytorch/ao pages convert to: #3604, 128x4 tiles in each group.) */
+mx_status mx_unrearrange_m_groups(const uint8_t *blocked, int64_t rows, int64_t cols,
+                                  const int32_t *group_end_offsets, int32_t num_groups, uint8_t *scales,
+                                  int64_t row_stride, cudaStream_t stream);
+
+/* Inverse of mx_rearrange_k_groups (groups along columns; uncovered columns
+ * at or past the last clamped end are written as 0). */
+mx_status mx_unrearrange_k_groups(const uint8_t *blocked, int64_t rows, int64_t cols,
+                                  const int32_t *group_end_offsets, int32_t num_groups, uint8_t *scales,
+                                  int64_t row_stride, cudaStream_t stream);
+
+/* Padded group starts as the blocked layout uses them (pytorch/ao #3285,
+ * Context: the new start of each padded group), for a consumer that would
+ * otherwise rescan: starts[g] = sum_{h<g} roundup(n_h, 128) rows (M) or
+ * sum_{h<g} roundup(w_h, 4) columns (K), and starts[G] = the padded total.
+ * `starts` is device int32[num_groups + 1]; one warp computes it on `stream`
+ * from the device offsets (clamped as above).  Group g's blocked bytes start
+ * at starts[g] * roundup(cols, 4) (M) or roundup(rows, 128) * starts[g] (K). */
+mx_status mx_padded_group_starts(mx_group_dim dim, int64_t rows, int64_t cols, const int32_t *group_end_offsets,
+                                 int32_t num_groups, int32_t *starts, cudaStream_t stream);
+
 /* The path AUTO would take for these arguments (host-only, no device access). */
 mx_path mx_select_path(mx_group_dim dim, const void *scales, int64_t rows, int64_t cols, int64_t row_stride);
 

@@ -13,14 +13,15 @@ from ._binding import (  # noqa: F401
     MX_GROUPS_K, MX_GROUPS_M, MX_MAX_GROUPS, MX_OK, MX_PATH_AUTO, MX_PATH_BYTE, MX_PATH_TMA,
     MX_PATH_WORD, PATHS, MxError, declared_symbols, lib, mx_device_flags, mx_rearrange_ex,
     mx_rearrange_k_groups, mx_rearrange_m_groups, mx_rearranged_size, mx_select_path,
-    mx_selftest_bounded_wait, mx_version,
-    status_string,
+    mx_padded_group_starts, mx_selftest_bounded_wait, mx_unrearrange_k_groups, mx_unrearrange_m_groups,
+    mx_version, status_string,
 )
 
 __all__ = [
     "rearrange_m_groups", "rearrange_k_groups", "rearrange", "rearranged_size",
     "mx_rearrange_m_groups", "mx_rearrange_k_groups", "mx_rearrange_ex", "mx_rearranged_size",
-    "mx_select_path", "mx_device_flags", "mx_version", "MxError",
+    "mx_select_path", "mx_device_flags", "mx_version", "MxError", "unrearrange", "padded_group_starts",
+    "mx_unrearrange_m_groups", "mx_unrearrange_k_groups", "mx_padded_group_starts",
 ]
 
 
@@ -72,3 +73,41 @@ def rearrange_m_groups(scales, group_end_offsets, out=None, path: str = "auto"):
 
 def rearrange_k_groups(scales, group_end_offsets, out=None, path: str = "auto"):
     return rearrange(MX_GROUPS_K, scales, group_end_offsets, out, path)
+
+
+def unrearrange(dim: int, blocked, rows: int, cols: int, group_end_offsets, out=None, stream=None):
+    """Inverse of ``rearrange``: the blocked flat uint8 buffer back to a
+    (rows, cols) uint8 tensor; elements no group covers come back as 0."""
+    import torch
+
+    if blocked.dtype != torch.uint8 or not blocked.is_contiguous() or not blocked.is_cuda:
+        raise ValueError("blocked must be a contiguous CUDA uint8 tensor")
+    if group_end_offsets.dtype != torch.int32 or not group_end_offsets.is_cuda:
+        raise ValueError("group_end_offsets must be a CUDA int32 tensor")
+    G = group_end_offsets.numel()
+    if blocked.numel() < mx_rearranged_size(dim, rows, cols, G):
+        raise ValueError("blocked is smaller than the layout's allocation")
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.uint8, device=blocked.device)
+    stride = out.stride(0) if rows > 1 else cols
+    if stream is None:
+        stream = torch.cuda.current_stream(blocked.device).cuda_stream
+    fn = mx_unrearrange_m_groups if dim == MX_GROUPS_M else mx_unrearrange_k_groups
+    st = fn(blocked.data_ptr(), rows, cols, group_end_offsets.data_ptr(), G, out.data_ptr(), stride, stream)
+    if st != MX_OK:
+        raise MxError("mx_unrearrange", st)
+    return out
+
+
+def padded_group_starts(dim: int, rows: int, cols: int, group_end_offsets, stream=None):
+    """int32[G + 1] padded group starts (rows for M, columns for K), computed on the GPU."""
+    import torch
+
+    G = group_end_offsets.numel()
+    starts = torch.empty(G + 1, dtype=torch.int32, device=group_end_offsets.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(group_end_offsets.device).cuda_stream
+    st = mx_padded_group_starts(dim, rows, cols, group_end_offsets.data_ptr(), G, starts.data_ptr(), stream)
+    if st != MX_OK:
+        raise MxError("mx_padded_group_starts", st)
+    return starts

@@ -37,6 +37,9 @@ _SIGNATURES = {
     "mx_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mx_device_flags": (ctypes.c_int, [_U32P, ctypes.c_int]),
     "mx_selftest_bounded_wait": (ctypes.c_int, [_I64, _P]),
+    "mx_unrearrange_m_groups": (ctypes.c_int, [_P, _I64, _I64, _P, _I32, _P, _I64, _P]),
+    "mx_unrearrange_k_groups": (ctypes.c_int, [_P, _I64, _I64, _P, _I32, _P, _I64, _P]),
+    "mx_padded_group_starts": (ctypes.c_int, [ctypes.c_int, _I64, _I64, _P, _I32, _P, _P]),
     "mx_version": (ctypes.c_int, []),
 }
 
@@ -94,6 +97,23 @@ def mx_rearrange_ex(dim: int, scales: int, rows: int, cols: int, row_stride: int
                     num_groups: int, out: int, path: int, stream: int) -> int:
     return lib().mx_rearrange_ex(dim, scales, rows, cols, row_stride, group_end_offsets, num_groups, out,
                                  path, stream)
+
+
+def mx_unrearrange_m_groups(blocked: int, rows: int, cols: int, group_end_offsets: int, num_groups: int,
+                            scales: int, row_stride: int, stream: int) -> int:
+    return lib().mx_unrearrange_m_groups(blocked, rows, cols, group_end_offsets, num_groups, scales, row_stride,
+                                         stream)
+
+
+def mx_unrearrange_k_groups(blocked: int, rows: int, cols: int, group_end_offsets: int, num_groups: int,
+                            scales: int, row_stride: int, stream: int) -> int:
+    return lib().mx_unrearrange_k_groups(blocked, rows, cols, group_end_offsets, num_groups, scales, row_stride,
+                                         stream)
+
+
+def mx_padded_group_starts(dim: int, rows: int, cols: int, group_end_offsets: int, num_groups: int, starts: int,
+                           stream: int) -> int:
+    return lib().mx_padded_group_starts(dim, rows, cols, group_end_offsets, num_groups, starts, stream)
 
 
 def mx_select_path(dim: int, scales: int, rows: int, cols: int, row_stride: int) -> int:

@@ -78,3 +78,27 @@ def test_status_strings(mxlib):
     for st in range(5):
         assert B.status_string(st)
     assert "misaligned" in B.status_string(B.MX_ERR_MISALIGNED)
+
+
+@pytest.mark.parametrize("kwargs,status", [
+    (dict(G=0), B.MX_ERR_INVALID_ARG),
+    (dict(G=65), B.MX_ERR_INVALID_ARG),
+    (dict(rows=-1), B.MX_ERR_INVALID_ARG),
+    (dict(stride=10), B.MX_ERR_INVALID_ARG),
+    (dict(ends=0), B.MX_ERR_INVALID_ARG),
+    (dict(blocked=0), B.MX_ERR_INVALID_ARG),
+    (dict(scales=0), B.MX_ERR_INVALID_ARG),
+    (dict(blocked=0x4004), B.MX_ERR_MISALIGNED),
+    (dict(rows=0), B.MX_OK),          # nothing to write, no launch
+])
+def test_inverse_host_validation(mxlib, kwargs, status):
+    a = dict(blocked=0x4000, rows=256, cols=64, ends=0x2000, G=2, scales=0x5000, stride=64)
+    a.update(kwargs)
+    for fn in (B.mx_unrearrange_m_groups, B.mx_unrearrange_k_groups):
+        assert fn(a["blocked"], a["rows"], a["cols"], a["ends"], a["G"], a["scales"], a["stride"], 0) == status
+
+
+def test_padded_starts_host_validation(mxlib):
+    assert B.mx_padded_group_starts(B.MX_GROUPS_M, 10, 10, 0, 2, 0x1000, 0) == B.MX_ERR_INVALID_ARG
+    assert B.mx_padded_group_starts(B.MX_GROUPS_M, 10, 10, 0x1000, 0, 0x2000, 0) == B.MX_ERR_INVALID_ARG
+    assert B.mx_padded_group_starts(7, 10, 10, 0x1000, 2, 0x2000, 0) == B.MX_ERR_INVALID_ARG

@@ -1,0 +1,96 @@
+"""GPU parity of the inverse rearrange (blocked -> row-major) and of the padded
+group starts, against the CPU oracle; round trips through both directions."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import scale_factor_layout_b200 as mxs  # noqa: E402
+from scale_factor_layout_b200 import _binding as B  # noqa: E402
+from scale_factor_layout_b200 import synth  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+SENTINEL = 0xEE
+
+
+def _inverse_check(case, orc, out_pad=0, misalign=0, blocked_np=None):
+    """Blocked input from the oracle (or given); run the GPU inverse into a
+    strided, possibly misaligned row-major buffer pre-filled with a sentinel."""
+    rows, cols, dim = case.rows, case.cols, case.dim
+    if blocked_np is None:
+        blocked_np = orc.rearrange(dim, case.scales, case.ends)
+    blocked = torch.from_numpy(blocked_np).cuda()
+    ends = torch.from_numpy(np.ascontiguousarray(case.ends, dtype=np.int32)).cuda()
+    stride = cols + out_pad
+    nbytes = rows * stride + misalign + 64
+    buf = torch.full((nbytes,), SENTINEL, dtype=torch.uint8, device="cuda")
+    ptr = buf.data_ptr() + misalign
+    fn = B.mx_unrearrange_m_groups if dim == synth.DIM_M else B.mx_unrearrange_k_groups
+    st = fn(blocked.data_ptr(), rows, cols, ends.data_ptr(), len(case.ends), ptr, stride,
+            torch.cuda.current_stream().cuda_stream)
+    assert st == B.MX_OK, B.status_string(st)
+    torch.cuda.synchronize()
+    host = buf.cpu().numpy()
+    assert (host[:misalign] == SENTINEL).all() and (host[misalign + rows * stride:] == SENTINEL).all()
+    view = host[misalign: misalign + rows * stride].reshape(rows, stride) if rows else np.zeros((0, stride), np.uint8)
+    want = orc.inverse(dim, blocked_np, rows, cols, case.ends)
+    if not np.array_equal(view[:, :cols], want):
+        bad = np.argwhere(view[:, :cols] != want)
+        raise AssertionError(f"{case.name}: {len(bad)} elements differ, first {bad[:5].tolist()}")
+    assert (view[:, cols:] == SENTINEL).all(), "row-stride gap bytes were written"
+
+
+@pytest.mark.parametrize("name", list(synth.NAMED))
+def test_inverse_workloads(mxlib, orc, name):
+    _inverse_check(synth.NAMED[name](), orc)
+
+
+@pytest.mark.parametrize("name,pad,misalign", [("m_tiny", 5, 3), ("m_wide", 16, 0), ("k_groups", 3, 1),
+                                               ("m_skinny", 4, 4), ("k_groups", 0, 8)])
+def test_inverse_strided_misaligned_out(mxlib, orc, name, pad, misalign):
+    _inverse_check(synth.NAMED[name](), orc, out_pad=pad, misalign=misalign)
+
+
+def test_inverse_sweep_subset(mxlib, orc):
+    for i_rows in range(len(synth.SWEEP_ROWS)):
+        for i_k in (0, 3, 6):
+            _inverse_check(synth.k_sweep_point(i_rows, i_k), orc)
+
+
+@pytest.mark.parametrize("chunk", range(4))
+def test_inverse_random_small(mxlib, orc, chunk):
+    for seed in range(500 + chunk * 50, 500 + chunk * 50 + 50):
+        c = synth.random_small(seed)
+        _inverse_check(c, orc, out_pad=seed % 7, misalign=seed % 5)
+
+
+def test_inverse_clamped_and_uncovered(mxlib, orc):
+    base = synth.m_tiny()
+    for ends in ([500, 300, 2000, 900], [0, 0, 0, 500], [100, 200, 300, 400]):
+        _inverse_check(synth.Case("clampM", synth.DIM_M, base.scales, np.asarray(ends, np.int32), 0), orc)
+        _inverse_check(synth.Case("clampK", synth.DIM_K, base.scales, np.asarray(ends, np.int32) // 20, 0), orc)
+
+
+def test_round_trip_on_gpu(mxlib, orc):
+    """forward then inverse on the GPU returns the covered input exactly."""
+    for c in (synth.m_wide(), synth.k_groups(), synth.m_skinny()):
+        s = torch.from_numpy(np.ascontiguousarray(c.scales)).cuda()
+        e = torch.from_numpy(c.ends).cuda()
+        blocked = mxs.rearrange(c.dim, s, e)
+        back = mxs.unrearrange(c.dim, blocked, c.rows, c.cols, e)
+        torch.cuda.synchronize()
+        assert torch.equal(back, s)
+
+
+def test_padded_group_starts(mxlib, orc):
+    rng = np.random.default_rng(17)
+    for _ in range(60):
+        dim = int(rng.integers(0, 2))
+        rows, cols, G = int(rng.integers(0, 20000)), int(rng.integers(1, 5000)), int(rng.integers(1, 65))
+        T = rows if dim == synth.DIM_M else cols
+        ends = rng.integers(-10, T + 50, size=G).astype(np.int32)
+        if rng.random() < 0.5:
+            ends = np.sort(ends)
+        got = mxs.padded_group_starts(dim, rows, cols, torch.from_numpy(ends).cuda()).cpu().numpy()
+        want = orc.padded_group_starts(dim, rows, cols, ends)
+        assert np.array_equal(got.astype(np.int64), want), (dim, rows, cols, ends)
