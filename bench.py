@@ -121,10 +121,13 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+FORWARD_SOURCES = ("mx_device.cuh", "mx_rearrange.cu")   # what the rearrange kernels are built from
+
+
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "scale_factor_layout_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in FORWARD_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -389,8 +392,8 @@ def run_ours(args, rank, world, local):
     dom = max(range(ncalls), key=lambda i: avg[i])
     dc = calls[dom]
     achieved = dc["read_bytes"] + dc["written_bytes"]
-    kernel_names = {"tma": "rearrange_tma", "flat": "rearrange_flat_tma", "word": "rearrange_fallback",
-                    "byte": "rearrange_fallback"}
+    kernel_names = {"tma": "rearrange_tma_m" if cases[dom].dim == 0 else "rearrange_tma_k",
+                    "flat": "rearrange_flat_tma", "word": "rearrange_fallback", "byte": "rearrange_fallback"}
     kname = "unrearrange_kernel" if args.op == "inverse" else kernel_names.get(dc["path"], "?")
     roofline = {"bound": "hbm", "kernel": f"{kname} ({dc['case']})",
                 "achieved": round(achieved / avg[dom] / 1e9, 1), "peak": peak, "unit": "GB/s",

@@ -349,6 +349,32 @@ __device__ __forceinline__ void read_rows_plain(const uint8_t *stage, int j, int
     }
 }
 
+// 16 bytes starting `off` bytes into a shared row (off + 32 within the row
+// when off is not a multiple of 16).
+__device__ __forceinline__ uint4 read16_at(const uint8_t *row, int off) {
+    const uint8_t *base = row + (off & ~15);
+    const uint4 lo = *reinterpret_cast<const uint4 *>(base);
+    if ((off & 15) == 0) return lo;
+    const uint4 hi = *reinterpret_cast<const uint4 *>(base + 16);
+    return realign(lo, hi, off & 15);
+}
+
+// 4 bytes starting `off` bytes into a shared row (off + 8 within the row).
+__device__ __forceinline__ uint32_t read4_at(const uint8_t *row, int off) {
+    const uint32_t *base = reinterpret_cast<const uint32_t *>(row + (off & ~3));
+    return __funnelshift_r(base[0], base[1], (off & 3) * 8);
+}
+
+// Index of group g with pstart[g] <= v < pstart[g + 1] (v < pstart[G]).
+__device__ __forceinline__ int find_group_pstart(const GroupTable &t, int G, int v) {
+    int lo = 0, hi = G;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (t.pstart[mid] <= v) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
 __device__ __forceinline__ uint32_t word_of(const uint4 &v, int t) {
     return t == 0 ? v.x : t == 1 ? v.y : t == 2 ? v.z : v.w;
 }

@@ -2,15 +2,18 @@
 // blocked layout on B200 (sm_100a).  Kernels and the C ABI of include/mxscale.h.
 //
 // Two kernels per grouping dimension:
-//   * rearrange_tma: persistent CTAs (one wave across the SMs); one thread
-//     streams 128-row boxes of scales into a ring of shared-memory stages with
-//     2-D TMA loads completed on mbarriers, while all 8 warps transpose the
-//     previous stages and store 512-byte tiles with 128-bit stores.  Needs the
-//     row stride to be a multiple of 16 bytes (the 2-D TMA stride rule named
-//     in pytorch/ao #3708, "fallback cuda kernel for when input doesn't meet
-//     2d TMA constraints", Context).
-//   * rearrange_fallback: the same work items loaded with ordinary 32-bit (or
-//     byte) loads, for any stride or alignment (#3708's fallback).
+//   * rearrange_tma_m / rearrange_tma_k: persistent CTAs (one wave across the
+//     SMs); one thread streams 128-row boxes of scales into a ring of
+//     shared-memory stages with 2-D TMA loads completed on mbarriers and
+//     writes finished tiles with bulk shared->global copies, while all 8 warps
+//     transpose the stages into staging blocks.  Needs the row stride to be a
+//     multiple of 16 bytes (the 2-D TMA stride rule named in pytorch/ao
+//     #3708, "fallback cuda kernel for when input doesn't meet 2d TMA
+//     constraints", Context).
+//   * rearrange_flat_tma: M-groups with narrow rows whose stride is a multiple
+//     of 4: 1-D TMA boxes over whole row blocks.
+//   * rearrange_fallback: work items loaded with ordinary 32-bit (or byte)
+//     loads, for any stride or alignment (#3708's fallback).
 // Every CTA scans the group ends itself (#3285, "compute prefix sum of group
 // sizes inside kernel", Changes), so no launch depends on device data known
 // to the host; the grid is sized from an upper bound on the work and CTAs
@@ -39,10 +42,13 @@ constexpr int kOutBytes = kTilesPerChunk * 512;
 template <bool kDimM>
 constexpr int stage_bytes() { return kDimM ? kStageBytesM : kStageBytesK; }
 
+// Dynamic shared memory of the M-groups (true) and K-groups (false) TMA kernels.
 template <bool kDimM>
 constexpr int tma_smem_bytes() { return kStages * stage_bytes<kDimM>() + kOutBuffers * kOutBytes + 1024; }
 
-// Persistent TMA kernel.  Per work item n of this CTA:
+// Persistent M-groups TMA kernel.  A work item is 128 rows x 128 columns of
+// one group (all columns of a row block in ceil(roundup(cols,4) / 128)
+// items), loaded as one 2-D box with 128-byte swizzle.  Per item n of a CTA:
 //   1. wait for its input box (stage n % kStages) and read 4 rows x 16 bytes
 //      per thread into registers;
 //   2. one barrier: the stage and the staging block n % 2 are free, and the
@@ -52,11 +58,10 @@ constexpr int tma_smem_bytes() { return kStages * stage_bytes<kDimM>() + kOutBuf
 //   4. every thread writes its masked output lines of item n into staging.
 // Loads and stores are both asynchronous copies driven by one thread, so the
 // 8 warps only move data between shared memory and registers.
-template <bool kDimM>
 __global__ void __launch_bounds__(kThreads, 2)
-rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restrict__ ends,
-              uint8_t *__restrict__ out, int64_t out_size, Shape s) {
-    constexpr int kStageBytes = stage_bytes<kDimM>();
+rearrange_tma_m(const __grid_constant__ CUtensorMap tmap, const int32_t *__restrict__ ends,
+                uint8_t *__restrict__ out, int64_t out_size, Shape s) {
+    constexpr int kStageBytes = kStageBytesM;
     extern __shared__ uint8_t dyn_smem[];
     // 128B swizzle needs 1024-byte aligned stage buffers
     uint8_t *stages = reinterpret_cast<uint8_t *>(
@@ -81,28 +86,26 @@ rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restric
     // placed as if no group were padded.  A prefetch has no observable value,
     // so it may run before the dependency wait.
     if (tid == 32) {
-        const int per_band = (s.cols + kChunkCols - 1) / kChunkCols + s.G / 2;
         for (int n = 0; n < kStages; ++n) {
             const int i = (int)blockIdx.x + n * (int)gridDim.x;
-            const int y = kDimM ? kTileRows * (i / s.col_chunks) : kTileRows * (i / per_band);
-            const int x = kDimM ? kChunkCols * (i % s.col_chunks)
-                                : min(kChunkCols * (i % per_band), s.cols - 1) & ~15;
+            const int y = kTileRows * (i / s.col_chunks);
+            const int x = kChunkCols * (i % s.col_chunks);
             if (y < s.rows) tma_prefetch_l2(&tmap, x, y);
         }
     }
     // Inputs may come from the previous kernel in the stream; outputs may
     // still be read by it.  No global load or store happens before this point.
     grid_dependency_wait();
-    if (q == 0) build_group_table<kDimM>(ends, s.G, kDimM ? s.rows : s.cols, s.col_chunks, table);
+    if (q == 0) build_group_table<true>(ends, s.G, s.rows, s.col_chunks, table);
     __syncthreads();
     grid_launch_dependents();
 
-    const int total = total_items<kDimM>(table, s);
+    const int total = total_items<true>(table, s);
     const int bid = blockIdx.x;
     const int n_my = bid < total ? (total - 1 - bid) / (int)gridDim.x + 1 : 0;
 
     auto issue = [&](int n, int st) {
-        const Item it = decode_item<kDimM>(table, s, bid + n * (int)gridDim.x, 16);
+        const Item it = decode_item<true>(table, s, bid + n * (int)gridDim.x, 16);
         items[st] = it;
         mbar_arrive_expect_tx(&full[st], kStageBytes);
         tma_load_2d(stages + st * kStageBytes, &tmap, it.x, it.y, &full[st]);
@@ -121,11 +124,7 @@ rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restric
         Item it;
         if (ok) {
             it = items[st];
-            const uint8_t *stage = stages + st * kStageBytes;
-            if (kDimM)
-                read_rows_swizzled(stage, j, q, w);
-            else
-                read_rows_plain(stage, j, q, it.delta, w);
+            read_rows_swizzled(stages + st * kStageBytes, j, q, w);
         }
         // the store that last read staging block n % 2 (item n-2) is the only
         // bulk group still outstanding here
@@ -159,7 +158,203 @@ rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restric
             bulk_commit();
         }
     }
-    zero_tail(out, covered_bytes<kDimM>(table, s), out_size);
+    zero_tail(out, covered_bytes<true>(table, s), out_size);
+    if (tid == 0) bulk_wait_all();
+}
+
+// K-groups TMA kernel.  A row band (128 rows) of the output holds, group
+// after group, each group's roundup(w_g, 4) / 4 tiles: the band's tile
+// stream.  A work item is a run of 32 consecutive tiles of that stream, so
+// only the band's last item is short, whatever the group sizes.  The 32
+// tiles' source columns span at most 128 input columns (a group boundary
+// skips back over the previous group's 0..3 padding columns), so one TMA box
+// 144 bytes wide, started at the 16-byte boundary below the first column,
+// holds the item.  A thread's 4 tiles usually lie in one group and are read
+// as one realigned 16-byte run per row; a quad that straddles a group
+// boundary reads each tile's 4 bytes on its own.  The item's tiles are
+// staged contiguously and written with one bulk store per group piece.
+struct KItem {
+    int32_t x, y;        // load origin (x a multiple of 16)
+    int32_t rows_valid;
+    int32_t tau0;        // first tile of the item in the band's tile stream
+    int32_t ntiles;
+    int32_t g0;          // group of tile tau0
+    int32_t rb;          // row band
+    int32_t pad;
+};
+
+__global__ void __launch_bounds__(kThreads, 2)
+rearrange_tma_k(const __grid_constant__ CUtensorMap tmap, const int32_t *__restrict__ ends,
+                uint8_t *__restrict__ out, int64_t out_size, Shape s) {
+    constexpr int kStageBytes = kStageBytesK;
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t *stages = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+    uint8_t *staging = stages + kStages * kStageBytes;
+    __shared__ GroupTable table;
+    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ KItem items[kStages];
+
+    const int tid = threadIdx.x;
+    const int j = tid & 31;
+    const int q = tid >> 5;
+
+    if (tid == 0) {
+        tma_prefetch_desc(&tmap);
+#pragma unroll
+        for (int st = 0; st < kStages; ++st) mbar_init(&full[st], 1);
+        fence_mbar_init();
+    }
+    // L2 prefetch of the boxes this CTA most likely loads first, placed as if
+    // no group were padded (no observable value, so before the wait).
+    if (tid == 32) {
+        const int per_band = (s.cols + kChunkCols - 1) / kChunkCols;
+        for (int n = 0; n < kStages; ++n) {
+            const int i = (int)blockIdx.x + n * (int)gridDim.x;
+            const int y = kTileRows * (i / per_band);
+            const int x = kChunkCols * (i % per_band);
+            if (y < s.rows) tma_prefetch_l2(&tmap, x, y);
+        }
+    }
+    grid_dependency_wait();
+    if (q == 0) build_group_table<false>(ends, s.G, s.cols, 1, table);
+    __syncthreads();
+    grid_launch_dependents();
+
+    const int T = table.pstart[kMaxGroups] >> 2;          // tiles per band
+    const int per_band = (T + kTilesPerChunk - 1) / kTilesPerChunk;
+    const int total = (s.padded_rows / kTileRows) * per_band;
+    const int bid = blockIdx.x;
+    const int n_my = bid < total ? (total - 1 - bid) / (int)gridDim.x + 1 : 0;
+
+    auto issue = [&](int n, int st) {
+        const int i = bid + n * (int)gridDim.x;
+        KItem it;
+        it.rb = i / per_band;
+        it.tau0 = (i - it.rb * per_band) * kTilesPerChunk;
+        it.ntiles = min(kTilesPerChunk, T - it.tau0);
+        it.g0 = find_group_pstart(table, s.G, 4 * it.tau0);
+        const int src0 = table.begin[it.g0] + 4 * it.tau0 - table.pstart[it.g0];
+        it.x = src0 & ~15;
+        it.y = it.rb * kTileRows;
+        it.rows_valid = min(kTileRows, s.rows - it.y);
+        it.pad = 0;
+        items[st] = it;
+        mbar_arrive_expect_tx(&full[st], kStageBytes);
+        tma_load_2d(stages + st * kStageBytes, &tmap, it.x, it.y, &full[st]);
+    };
+
+    // Thread 0 writes the staged tiles of an item, one bulk copy per group piece.
+    auto store_item = [&](const KItem &it, const uint8_t *stg) {
+        int g = it.g0;
+        for (int t = 0; t < it.ntiles;) {
+            const int tau = it.tau0 + t;
+            while (table.pstart[g + 1] <= 4 * tau) ++g;
+            const int end = min(it.tau0 + it.ntiles, table.pstart[g + 1] >> 2);
+            const int W = table.pstart[g + 1] - table.pstart[g];
+            const int64_t dst = (int64_t)s.padded_rows * table.pstart[g] + (int64_t)it.rb * kTileRows * W +
+                                (int64_t)(tau - (table.pstart[g] >> 2)) * 512;
+            bulk_store_s2g(out + dst, stg + t * 512, (uint32_t)(end - tau) * 512u);
+            t = end - it.tau0;
+            ++g;
+        }
+        bulk_commit();
+    };
+
+    if (tid == 0)
+        for (int st = 0; st < kStages && st < n_my; ++st) issue(st, st);
+
+    KItem prev;
+    prev.ntiles = 0;
+    for (int n = 0; n < n_my; ++n) {
+        const int st = n % kStages;
+        const uint32_t parity = (uint32_t)(n / kStages) & 1u;
+        const bool ok = mbar_wait_bounded(&full[st], parity);
+        uint4 w[4] = {};
+        uint32_t cm[4] = {0u, 0u, 0u, 0u};
+        KItem it;
+        if (ok) {
+            it = items[st];
+            const uint8_t *stage = stages + st * kStageBytes;
+            const int tl0 = 4 * q;
+            if (tl0 < it.ntiles) {
+                const int tau = it.tau0 + tl0;
+                int g = it.g0;
+                while (table.pstart[g + 1] <= 4 * tau) ++g;
+                const int last = min(tl0 + 3, it.ntiles - 1);
+                const int src = table.begin[g] + 4 * tau - table.pstart[g];
+                if (4 * (it.tau0 + last) < table.pstart[g + 1]) {
+                    // the quad's tiles are consecutive columns of one group
+                    const int gend = table.begin[g] + table.size[g];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const int nv = tl0 + t < it.ntiles ? gend - (src + 4 * t) : 0;
+                        cm[t] = nv >= 4 ? 0xffffffffu : (nv <= 0 ? 0u : ((1u << (8 * nv)) - 1u));
+                    }
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+                        w[a] = read16_at(stage + (j + 32 * a) * kPitchPlain, src - it.x);
+                } else {
+                    // the quad crosses into a later group: one tile at a time
+                    int gt = g;
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const int tl = tl0 + t;
+                        if (tl < it.ntiles) {
+                            while (table.pstart[gt + 1] <= 4 * (it.tau0 + tl)) ++gt;
+                            const int srct = table.begin[gt] + 4 * (it.tau0 + tl) - table.pstart[gt];
+                            const int nv = table.begin[gt] + table.size[gt] - srct;
+                            cm[t] = nv >= 4 ? 0xffffffffu : ((1u << (8 * nv)) - 1u);
+#pragma unroll
+                            for (int a = 0; a < 4; ++a) {
+                                const uint32_t v = read4_at(stage + (j + 32 * a) * kPitchPlain, srct - it.x);
+                                if (t == 0) w[a].x = v; else if (t == 1) w[a].y = v; else if (t == 2) w[a].z = v; else w[a].w = v;
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        if (tid == 0) bulk_wait_read<0>();
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_mx_flags, kFlagWaitTimeout);
+                for (int m = n; m < n_my && m < n + kStages; ++m)
+                    mbar_wait_bounded(&full[m % kStages], (uint32_t)(m / kStages) & 1u);
+            }
+            return;
+        }
+        if (tid == 0) {
+            if (n > 0) store_item(prev, staging + ((n - 1) & 1) * kOutBytes);
+            prev = it;
+            if (n + kStages < n_my) issue(n + kStages, st);
+        }
+        // masked lines of this thread's tiles into staging block n % 2
+        {
+            uint8_t *stg = staging + (n & 1) * kOutBytes;
+            uint32_t rm[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) rm[a] = (j + 32 * a < it.rows_valid) ? 0xffffffffu : 0u;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int tl = 4 * q + t;
+                if (tl < it.ntiles) {
+                    uint4 o;
+                    o.x = word_of(w[0], t) & rm[0] & cm[t];
+                    o.y = word_of(w[1], t) & rm[1] & cm[t];
+                    o.z = word_of(w[2], t) & rm[2] & cm[t];
+                    o.w = word_of(w[3], t) & rm[3] & cm[t];
+                    *reinterpret_cast<uint4 *>(stg + tl * 512 + 16 * j) = o;
+                }
+            }
+        }
+        fence_proxy_async_smem();
+    }
+    if (n_my > 0) {
+        __syncthreads();
+        if (tid == 0) store_item(prev, staging + ((n_my - 1) & 1) * kOutBytes);
+    }
+    zero_tail(out, (int64_t)s.padded_rows * table.pstart[kMaxGroups], out_size);
     if (tid == 0) bulk_wait_all();
 }
 
@@ -171,7 +366,7 @@ rearrange_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restric
 // 16-byte boundary at or below its first byte (boxes past the array's end
 // read zeros).  Rows sit at pitch row_stride in shared memory; with the
 // stride a multiple of 4 every row starts on a word, and the transpose reads
-// 32-bit words.  Pipeline, staging and bulk stores follow rearrange_tma.
+// 32-bit words.  Pipeline, staging and bulk stores follow rearrange_tma_m.
 constexpr int kFlatBoxWords = 256;
 constexpr int kFlatBoxBytes = kFlatBoxWords * 4;
 constexpr int kFlatStages = 4;
@@ -462,14 +657,14 @@ mx_status device_info(const DeviceInfo **out) {
         const int flat_max = flat_smem_bytes(flat_shape(kFlatMaxStride, kFlatMaxStride));
         if (cudaFuncSetAttribute(rearrange_flat_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, flat_max) !=
                 cudaSuccess ||
-            cudaFuncSetAttribute(rearrange_tma<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(rearrange_tma_m, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tma_smem_bytes<true>()) != cudaSuccess ||
-            cudaFuncSetAttribute(rearrange_tma<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(rearrange_tma_k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tma_smem_bytes<false>()) != cudaSuccess)
             return MX_ERR_CUDA;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_tma[1], rearrange_tma<true>, kThreads,
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_tma[1], rearrange_tma_m, kThreads,
                                                           tma_smem_bytes<true>()) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_tma[0], rearrange_tma<false>, kThreads,
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_tma[0], rearrange_tma_k, kThreads,
                                                           tma_smem_bytes<false>()) != cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_fallback, rearrange_fallback<true, true>,
                                                           kThreads, 0) != cudaSuccess)
@@ -583,9 +778,9 @@ mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t col
         const int64_t cap = (int64_t)d->sms * d->occ_tma[dim_m ? 1 : 0];
         const int grid = (int)(work < cap ? work : cap);
         if (dim_m)
-            launch_pdl(rearrange_tma<true>, grid, tma_smem_bytes<true>(), stream, map, ends, out, (int64_t)size, s);
+            launch_pdl(rearrange_tma_m, grid, tma_smem_bytes<true>(), stream, map, ends, out, (int64_t)size, s);
         else
-            launch_pdl(rearrange_tma<false>, grid, tma_smem_bytes<false>(), stream, map, ends, out, (int64_t)size, s);
+            launch_pdl(rearrange_tma_k, grid, tma_smem_bytes<false>(), stream, map, ends, out, (int64_t)size, s);
     } else if (path == MX_PATH_FLAT) {
         auto encode = encode_fn();
         if (encode == nullptr) return MX_ERR_CUDA;
