@@ -358,10 +358,26 @@ def run_ours(args, rank, world, local):
         barrier(dist, device)
         return start.elapsed_time(end) / 1e3
 
+    def capture_copies(i):
+        """The practical ceiling for call i: a D2D copy of its input bytes
+        (read + write the same traffic), same rotation, same graph timing."""
+        srcs = [it[1] for it in rot[i]]
+        dsts = [torch.empty_like(x) for x in srcs]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            for a, b in zip(srcs, dsts):   # warm the copy path outside capture
+                b.copy_(a)
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                for k in range(args.steps):
+                    dsts[k % len(dsts)].copy_(srcs[k % len(srcs)])
+        return g, dsts
+
     warm_g = capture(steps_of(0, args.warmup))
     timed_g = capture(steps_of(args.warmup, args.steps))
     # each call on its own: the same launches back to back, one call type per graph
     per_call_g = [capture([rot[i][k % len(rot[i])] for k in range(args.steps)]) for i in range(ncalls)]
+    copy_g = [capture_copies(i) for i in range(ncalls)] if not args.no_copy_ceiling else None
 
     sampler = ClockSampler(local)
     with sampler:
@@ -376,19 +392,31 @@ def run_ours(args, rank, world, local):
             with torch.cuda.stream(stream):
                 warm_g.replay()
             avg.append(max_over_ranks(replay_timed(g), dist, device) / args.steps)
+        copy_avg = None
+        if copy_g is not None:
+            copy_avg = []
+            for g, _ in copy_g:
+                with torch.cuda.stream(stream):
+                    warm_g.replay()
+                copy_avg.append(max_over_ranks(replay_timed(g), dist, device) / args.steps)
     seconds_max = max_over_ranks(seconds, dist, device)
-    del timed_g, warm_g, per_call_g
+    del timed_g, warm_g, per_call_g, copy_g
 
     peak, peak_src = load_peaks()
     value = aggregate_value(step_bytes, args.steps, world, seconds_max)
     calls = []
-    for c, b, t in zip(cases, per_call, avg):
+    for ci, (c, b, t) in enumerate(zip(cases, per_call, avg)):
         gbs = (b["read"] + b["written"]) / t / 1e9
         path = mxs.mx_select_path(c.dim, rot[cases.index(c)][0][1].data_ptr(), c.rows, c.cols, c.cols)
         calls.append({"case": c.name, "path": B.PATH_NAMES.get(path, "?"),
                       "us": round(t * 1e6, 3), "gbps": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
                       "read_bytes": b["read"], "written_bytes": b["written"], "alloc_bytes": b["alloc"],
                       "gbps_pages_convention": round((b["read"] + b["alloc"]) / t / 1e9, 1)})
+        if copy_avg is not None:
+            cbytes = 2 * c.rows * c.cols   # the copy reads and writes the input's bytes
+            cg = cbytes / copy_avg[ci] / 1e9
+            calls[-1].update({"copy_us": round(copy_avg[ci] * 1e6, 3), "copy_gbps": round(cg, 1),
+                              "frac_of_copy": round(gbs / cg, 4)})
     dom = max(range(ncalls), key=lambda i: avg[i])
     dc = calls[dom]
     achieved = dc["read_bytes"] + dc["written_bytes"]
@@ -577,6 +605,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-copy-ceiling", action="store_true",
+                    help="skip timing a same-size device-to-device copy per call")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)

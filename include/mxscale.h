@@ -46,7 +46,8 @@
  * that first call before any stream capture.  Calls are thread-safe.
  *
  * Errors.  Argument faults the host can see return a status and launch
- * nothing.  A launch failure returns MX_ERR_CUDA (from cudaGetLastError).
+ * nothing.  A failed CUDA call returns MX_ERR_CUDA (mx_last_cuda_error gives
+ * the CUDA code).
  * Bad device-side offsets are clamped as stated above.
  */
 #ifndef MXSCALE_H
@@ -163,6 +164,11 @@ mx_status mx_device_flags(uint32_t *flags, int clear);
  * of the device flags; read them with mx_device_flags.  The kernel returns
  * normally and the context stays usable.  Asynchronous on `stream`. */
 mx_status mx_selftest_bounded_wait(int64_t limit_cycles, cudaStream_t stream);
+
+/* The CUDA error code behind the calling thread's most recent MX_ERR_CUDA
+ * (0 if none): a cudaError_t, or the CUresult of a failed tensor-map encode.  The library reports launch failures from the launch's own
+ * return code and never reads or clears the thread's pending CUDA error. */
+int mx_last_cuda_error(void);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int mx_version(void);

@@ -40,13 +40,15 @@ _SIGNATURES = {
     "mx_unrearrange_m_groups": (ctypes.c_int, [_P, _I64, _I64, _P, _I32, _P, _I64, _P]),
     "mx_unrearrange_k_groups": (ctypes.c_int, [_P, _I64, _I64, _P, _I32, _P, _I64, _P]),
     "mx_padded_group_starts": (ctypes.c_int, [ctypes.c_int, _I64, _I64, _P, _I32, _P, _P]),
+    "mx_last_cuda_error": (ctypes.c_int, []),
     "mx_version": (ctypes.c_int, []),
 }
 
 
 class MxError(RuntimeError):
     def __init__(self, where: str, status: int):
-        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        extra = f", CUDA error {mx_last_cuda_error()}" if status == MX_ERR_CUDA else ""
+        super().__init__(f"{where}: {status_string(status)} (status {status}{extra})")
         self.status = status
 
 
@@ -130,6 +132,10 @@ def mx_device_flags(clear: bool = False) -> int:
 
 def mx_selftest_bounded_wait(limit_cycles: int, stream: int = 0) -> int:
     return lib().mx_selftest_bounded_wait(limit_cycles, stream)
+
+
+def mx_last_cuda_error() -> int:
+    return int(lib().mx_last_cuda_error())
 
 
 def mx_version() -> int:

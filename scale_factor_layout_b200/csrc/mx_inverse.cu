@@ -16,6 +16,9 @@
 #include "mx_device.cuh"
 #include "mxscale.h"
 
+// Defined in mx_rearrange.cu: note a CUDA failure for mx_last_cuda_error().
+mx_status mx_record_cuda_error(cudaError_t e);
+
 namespace mx {
 namespace {
 
@@ -175,16 +178,16 @@ mx_status unrearrange(mx_group_dim dim, const uint8_t *blocked, int64_t rows, in
                                 : ceil_div(rows, 128) * (ceil_div(cols, kChunkCols) + G);
     if (bound > INT_MAX) return MX_ERR_UNSUPPORTED;
     int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return MX_ERR_CUDA;
+    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return mx_record_cuda_error(e);
+    if (cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev); e != cudaSuccess)
+        return mx_record_cuda_error(e);
     const int64_t cap = (int64_t)sms * 8 * 4;
     const int grid = (int)(bound < 1 ? 1 : (bound < cap ? bound : cap));
     cudaError_t e = dim_m ? launch_pdl(unrearrange_kernel<true>, grid, kThreads, stream, blocked, ends, scales,
                                        row_stride, s)
                           : launch_pdl(unrearrange_kernel<false>, grid, kThreads, stream, blocked, ends, scales,
                                        row_stride, s);
-    return e == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+    return e == cudaSuccess ? MX_OK : mx_record_cuda_error(e);
 }
 
 }  // namespace
@@ -216,7 +219,7 @@ mx_status mx_padded_group_starts(mx_group_dim dim, int64_t rows, int64_t cols, c
     cudaError_t e = dim == MX_GROUPS_M
                         ? mx::launch_pdl(mx::padded_starts_kernel<true>, 1, 32, stream, group_end_offsets, starts, s)
                         : mx::launch_pdl(mx::padded_starts_kernel<false>, 1, 32, stream, group_end_offsets, starts, s);
-    return e == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+    return e == cudaSuccess ? MX_OK : mx_record_cuda_error(e);
 }
 
 }  // extern "C"

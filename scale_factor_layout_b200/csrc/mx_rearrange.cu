@@ -631,6 +631,15 @@ FlatShape flat_shape(int64_t row_stride, int64_t padded_cols) {
 
 int flat_smem_bytes(const FlatShape &f) { return kFlatStages * f.stage_bytes + 2 * f.staging_bytes + 128; }
 
+// The CUDA error behind the calling thread's latest MX_ERR_CUDA.
+thread_local cudaError_t t_last_error = cudaSuccess;
+
+mx_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return MX_OK;
+    t_last_error = e;
+    return MX_ERR_CUDA;
+}
+
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -649,27 +658,35 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 mx_status device_info(const DeviceInfo **out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MX_ERR_CUDA;
+    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
+    if (dev < 0 || dev >= kMaxDevices) return MX_ERR_UNSUPPORTED;
+    // The tensor-map encoder is a driver call and needs the device's primary
+    // context current in this thread; a thread whose first CUDA work is this
+    // call has none yet, so bind it once per thread and device.
+    thread_local int t_bound_dev = -1;
+    if (t_bound_dev != dev) {
+        if (cudaError_t e = cudaSetDevice(dev); e != cudaSuccess) return cuda_status(e);
+        t_bound_dev = dev;
+    }
     std::lock_guard<std::mutex> lock(g_mu);
     DeviceInfo &d = g_dev[dev];
     if (!d.ready) {
-        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MX_ERR_CUDA;
+        if (cudaError_t e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev); e != cudaSuccess)
+            return cuda_status(e);
         const int flat_max = flat_smem_bytes(flat_shape(kFlatMaxStride, kFlatMaxStride));
-        if (cudaFuncSetAttribute(rearrange_flat_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, flat_max) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(rearrange_tma_m, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tma_smem_bytes<true>()) != cudaSuccess ||
-            cudaFuncSetAttribute(rearrange_tma_k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tma_smem_bytes<false>()) != cudaSuccess)
-            return MX_ERR_CUDA;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_tma[1], rearrange_tma_m, kThreads,
-                                                          tma_smem_bytes<true>()) != cudaSuccess ||
+        const cudaError_t setup[] = {
+            cudaFuncSetAttribute(rearrange_flat_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, flat_max),
+            cudaFuncSetAttribute(rearrange_tma_m, cudaFuncAttributeMaxDynamicSharedMemorySize, tma_smem_bytes<true>()),
+            cudaFuncSetAttribute(rearrange_tma_k, cudaFuncAttributeMaxDynamicSharedMemorySize, tma_smem_bytes<false>()),
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_tma[1], rearrange_tma_m, kThreads,
+                                                          tma_smem_bytes<true>()),
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_tma[0], rearrange_tma_k, kThreads,
-                                                          tma_smem_bytes<false>()) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_fallback, rearrange_fallback<true, true>,
-                                                          kThreads, 0) != cudaSuccess)
-            return MX_ERR_CUDA;
-        if (d.occ_tma[0] < 1 || d.occ_tma[1] < 1 || d.occ_fallback < 1) return MX_ERR_CUDA;
+                                                          tma_smem_bytes<false>()),
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_fallback, rearrange_fallback<true, true>, kThreads, 0),
+        };
+        for (cudaError_t e : setup)
+            if (e != cudaSuccess) return cuda_status(e);
+        if (d.occ_tma[0] < 1 || d.occ_tma[1] < 1 || d.occ_fallback < 1) return cuda_status(cudaErrorInvalidConfiguration);
         d.ready = true;
     }
     *out = &d;
@@ -680,7 +697,7 @@ mx_status device_info(const DeviceInfo **out) {
 // while the previous kernel in the stream drains; it waits for that kernel's
 // completion (griddepcontrol.wait) before touching global memory.
 template <typename... KArgs, typename... Args>
-void launch_pdl(void (*kernel)(KArgs...), int grid, int smem, cudaStream_t stream, Args... args) {
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int smem, cudaStream_t stream, Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
@@ -691,7 +708,7 @@ void launch_pdl(void (*kernel)(KArgs...), int grid, int smem, cudaStream_t strea
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -761,10 +778,11 @@ mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t col
     const DeviceInfo *d = nullptr;
     if (mx_status st = device_info(&d); st != MX_OK) return st;
     const int64_t work = bound > 0 ? bound : 1;
+    cudaError_t launched = cudaSuccess;
 
     if (path == MX_PATH_TMA) {
         auto encode = encode_fn();
-        if (encode == nullptr) return MX_ERR_CUDA;
+        if (encode == nullptr) return cuda_status(cudaErrorSymbolNotFound);
         CUtensorMap map;
         cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
         cuuint64_t gstride[1] = {(cuuint64_t)row_stride};
@@ -774,16 +792,16 @@ mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t col
                             box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                             dim_m ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return MX_ERR_CUDA;
+        if (r != CUDA_SUCCESS) return cuda_status(static_cast<cudaError_t>(r));   // driver code
         const int64_t cap = (int64_t)d->sms * d->occ_tma[dim_m ? 1 : 0];
         const int grid = (int)(work < cap ? work : cap);
-        if (dim_m)
-            launch_pdl(rearrange_tma_m, grid, tma_smem_bytes<true>(), stream, map, ends, out, (int64_t)size, s);
-        else
-            launch_pdl(rearrange_tma_k, grid, tma_smem_bytes<false>(), stream, map, ends, out, (int64_t)size, s);
+        launched = dim_m ? launch_pdl(rearrange_tma_m, grid, tma_smem_bytes<true>(), stream, map, ends, out,
+                                      (int64_t)size, s)
+                         : launch_pdl(rearrange_tma_k, grid, tma_smem_bytes<false>(), stream, map, ends, out,
+                                      (int64_t)size, s);
     } else if (path == MX_PATH_FLAT) {
         auto encode = encode_fn();
-        if (encode == nullptr) return MX_ERR_CUDA;
+        if (encode == nullptr) return cuda_status(cudaErrorSymbolNotFound);
         CUtensorMap map;
         cuuint64_t gdim[1] = {(cuuint64_t)(((rows - 1) * row_stride + cols) / 4)};
         cuuint64_t gstride[1] = {0};
@@ -792,28 +810,31 @@ mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t col
         CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 1, const_cast<uint8_t *>(scales), gdim, gstride,
                             box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return MX_ERR_CUDA;
+        if (r != CUDA_SUCCESS) return cuda_status(static_cast<cudaError_t>(r));   // driver code
         const FlatShape f = flat_shape(row_stride, s.padded_cols);
         const int smem = flat_smem_bytes(f);
         int occ = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rearrange_flat_tma, kThreads, smem) != cudaSuccess ||
-            occ < 1)
-            return MX_ERR_CUDA;
+        if (cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rearrange_flat_tma, kThreads, smem);
+            e != cudaSuccess || occ < 1)
+            return cuda_status(e != cudaSuccess ? e : cudaErrorInvalidConfiguration);
         const int64_t cap = (int64_t)d->sms * occ;
         const int grid = (int)(work < cap ? work : cap);
-        launch_pdl(rearrange_flat_tma, grid, smem, stream, map, ends, out, (int64_t)size, s, f);
+        launched = launch_pdl(rearrange_flat_tma, grid, smem, stream, map, ends, out, (int64_t)size, s, f);
     } else {
         const int64_t cap = (int64_t)d->sms * d->occ_fallback * 4;
         const int grid = (int)(work < cap ? work : cap);
         const bool word = path == MX_PATH_WORD;
         auto kernel = dim_m ? (word ? rearrange_fallback<true, true> : rearrange_fallback<true, false>)
                             : (word ? rearrange_fallback<false, true> : rearrange_fallback<false, false>);
-        launch_pdl(kernel, grid, 0, stream, scales, row_stride, ends, out, (int64_t)size, s);
+        launched = launch_pdl(kernel, grid, 0, stream, scales, row_stride, ends, out, (int64_t)size, s);
     }
-    return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+    return cuda_status(launched);
 }
 
 }  // namespace mx
+
+// Shared with mx_inverse.cu (C++ linkage, not part of the C ABI).
+mx_status mx_record_cuda_error(cudaError_t e) { return mx::cuda_status(e); }
 
 // ------------------------------------------------------------------ C ABI
 extern "C" {
@@ -864,20 +885,25 @@ const char *mx_status_string(mx_status status) {
 mx_status mx_device_flags(uint32_t *flags, int clear) {
     if (flags == nullptr) return MX_ERR_INVALID_ARG;
     unsigned int v = 0;
-    if (cudaMemcpyFromSymbol(&v, mx::g_mx_flags, sizeof(v)) != cudaSuccess) return MX_ERR_CUDA;
+    if (cudaError_t e = cudaMemcpyFromSymbol(&v, mx::g_mx_flags, sizeof(v)); e != cudaSuccess)
+        return mx::cuda_status(e);
     *flags = v;
     if (clear) {
         const unsigned int zero = 0;
-        if (cudaMemcpyToSymbol(mx::g_mx_flags, &zero, sizeof(zero)) != cudaSuccess) return MX_ERR_CUDA;
+        if (cudaError_t e = cudaMemcpyToSymbol(mx::g_mx_flags, &zero, sizeof(zero)); e != cudaSuccess)
+            return mx::cuda_status(e);
     }
     return MX_OK;
 }
 
 mx_status mx_selftest_bounded_wait(int64_t limit_cycles, cudaStream_t stream) {
     if (limit_cycles < 1 || limit_cycles > (1ll << 32)) return MX_ERR_INVALID_ARG;
-    mx::bounded_wait_selftest<<<1, 32, 0, stream>>>((long long)limit_cycles);
-    return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+    void *args[] = {&limit_cycles};
+    return mx::cuda_status(cudaLaunchKernel(reinterpret_cast<const void *>(mx::bounded_wait_selftest), dim3(1),
+                                            dim3(32), args, 0, stream));
 }
+
+int mx_last_cuda_error(void) { return (int)mx::t_last_error; }
 
 int mx_version(void) { return 100; }
 
