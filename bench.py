@@ -122,15 +122,20 @@ def load_peaks():
 
 
 FORWARD_SOURCES = ("mx_device.cuh", "mx_rearrange.cu")   # what the rearrange kernels are built from
+HOST_MARKER = b"// ------------------------------------------------------------------ host side"
 
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(root: str = ROOT) -> str:
+    """sha256 prefix of the forward kernels' device code (mx_device.cuh, and
+    mx_rearrange.cu up to its host-side section)."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "scale_factor_layout_b200", "csrc")
+    csrc = os.path.join(root, "scale_factor_layout_b200", "csrc")
     for name in FORWARD_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode())
-            h.update(f.read())
+            data = f.read()
+        cut = data.find(HOST_MARKER)
+        h.update(name.encode())
+        h.update(data if cut < 0 else data[:cut])
     return h.hexdigest()[:16]
 
 
