@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include <climits>
+#include <mutex>
 
 #include "mx_device.cuh"
 #include "mxscale.h"
@@ -22,88 +23,274 @@ mx_status mx_record_cuda_error(cudaError_t e);
 namespace mx {
 namespace {
 
-// Shared-memory row block of one work item: 128 rows x 128 columns at pitch
-// 176 bytes (11 x 16, odd: conflict-free 16-byte accesses down a column),
-// the item's first column 16 bytes into each row so that a window may start
-// up to 15 bytes before it.
-constexpr int kInvPitch = 176;
-constexpr int kInvLead = 16;
-constexpr int kInvChunks = 9;   // 16-byte global chunks a 128-column row segment can touch
+// 1-D bulk copy global -> shared (16-byte aligned addresses, bytes a multiple
+// of 16), completed on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_load_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
 
-// One CTA per work item (grid-stride).
-//  1. Thread (j = lane, q = warp) loads line j of tiles 4q..4q+3 (a warp reads
-//     one whole 512-byte tile per 128-bit load); word a of line j of tile cb
-//     holds row j + 32a, columns 4cb .. 4cb+3, so a 4x4 word transpose in
-//     registers gives 16 bytes of each of rows j, j+32, j+64, j+96, which go to
-//     the shared row block.
-//  2. Threads then walk (row, 16-byte-aligned global chunk) pairs: each reads
-//     the 32-byte shared window around its chunk, shifts it into place, and
-//     stores 16 bytes (or only the bytes of the item at a row's head and tail).
+// Bring `bytes` (a multiple of 16) of global memory at a 16-byte aligned
+// address into L2 only.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
+
+// Shared-memory row block of one work item: 128 rows of up to 36 tiles' columns
+// (the item's 32 tiles and the quad before them) at pitch 144 bytes (9 x 16,
+// odd: conflict-free 16-byte accesses down a column).  In flat mode the rows
+// sit back to back instead (row r at r * cols).
+constexpr int kInvPreTiles = 4;                                         // quad loaded before an item
+constexpr int kInvPitch = (kTilesPerChunk + kInvPreTiles) * 4;          // 144
+constexpr int kInvStages = 2;                                           // items in flight per CTA
+constexpr int kInvStageBytes = (kTilesPerChunk + kInvPreTiles) * 512;   // 18 KB
+constexpr int kInvBlockBytes = kTileRows * kInvPitch;                   // 18 KB
+constexpr int kInvSmemBytes = kInvStages * kInvStageBytes + 2 * kInvBlockBytes + 128;
+constexpr uint32_t kInvFlagWaitTimeout = 1u;
+
+// Error flags of the inverse kernels (a pipeline wait ran past its limit).
+__device__ unsigned int g_inv_flags = 0;
+
+// A work item of the inverse.  Output columns of one row are written by
+// whole 16-byte-aligned chunks; a chunk that straddles two items of the same
+// run (a group's columns for K, a row's columns for M) belongs to the later
+// item, which therefore also loads the quad of tiles just before its own
+// (contiguous in the blocked buffer).  Partial chunks remain only where a
+// run starts or ends.
+struct InvItem {
+    int64_t src_off;      // blocked offset of the first tile loaded
+    int32_t x, y;         // first output column and row of the item
+    int32_t rows_valid;   // rows with data
+    int32_t ncol;         // item columns with data (<= 128)
+    int32_t nload;        // tiles loaded (own, plus the previous quad)
+    int32_t pre;          // columns before the item's first one in the stage: 0 or 16
+    int32_t last;         // 1 if the item ends its run
+    int32_t pad;
+};
+
+// `out`, `row_stride`: the row-major output, to tell whether an item's first
+// column can start mid-chunk (only then is the quad before it needed).
 template <bool kDimM>
-__global__ void __launch_bounds__(kThreads)
-unrearrange_kernel(const uint8_t *__restrict__ blocked, const int32_t *__restrict__ ends,
-                   uint8_t *__restrict__ scales, int64_t row_stride, Shape s) {
+__device__ __forceinline__ InvItem decode_inv(const GroupTable &t, const Shape &s, int i, const uint8_t *out,
+                                              int64_t row_stride) {
+    const Item it = decode_item<kDimM>(t, s, i, 1);
+    int k, run;   // item's chunk index in its run, and the run's column count
+    if (kDimM) {
+        const int g = find_group(t, s.G, i);
+        const int local = i - t.istart[g];
+        k = local - (local / s.col_chunks) * s.col_chunks;
+        run = s.cols;
+    } else {
+        const int per_band = t.istart[kMaxGroups];
+        const int local = i - (i / per_band) * per_band;
+        const int g = find_group(t, s.G, local);
+        k = local - t.istart[g];
+        run = t.size[g];
+    }
+    // every row of the item starts 16-byte aligned: no chunk straddles the
+    // item's first column, so nothing before it is needed
+    const bool aligned = (row_stride & 15) == 0 &&
+                         ((reinterpret_cast<uintptr_t>(out + (int64_t)it.y * row_stride + it.x) & 15u) == 0);
+    const bool pre = k > 0 && !aligned;
+    InvItem v;
+    v.x = it.x;
+    v.y = it.y;
+    v.rows_valid = it.rows_valid;
+    v.ncol = it.cols_valid;
+    v.pre = pre ? 4 * kInvPreTiles : 0;
+    v.nload = it.ntiles + (pre ? kInvPreTiles : 0);
+    v.src_off = it.out_off - (pre ? kInvPreTiles * 512 : 0);
+    v.last = kTilesPerChunk * 4 * (k + 1) >= run ? 1 : 0;
+    v.pad = 0;
+    return v;
+}
+
+// 16 bytes starting at byte o of a shared row (o may be negative; bytes
+// outside [0, limit) read as zero).
+__device__ __forceinline__ uint4 window16(const uint8_t *row, int o, int limit) {
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    const int f = o & ~15;
+    const int d = o - f;
+    const uint4 lo = (f >= 0 && f < limit) ? *reinterpret_cast<const uint4 *>(row + f) : zero;
+    if (d == 0) return lo;
+    const uint4 hi = (f + 16 >= 0 && f + 16 < limit) ? *reinterpret_cast<const uint4 *>(row + f + 16) : zero;
+    return realign(lo, hi, d);
+}
+
+// Store bytes [kmin, kmax) of v at the 16-byte aligned dst.
+__device__ __forceinline__ void store16_part(uint8_t *dst, const uint4 &v, int kmin, int kmax) {
+    if (kmin == 0 && kmax == 16) {
+        *reinterpret_cast<uint4 *>(dst) = v;
+        return;
+    }
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) {
+        const int b0 = 4 * k4;
+        if (b0 >= kmin && b0 + 4 <= kmax) {
+            *reinterpret_cast<uint32_t *>(dst + b0) = wv[k4];
+        } else {
+            for (int b = max(b0, kmin); b < min(b0 + 4, kmax); ++b) dst[b] = (uint8_t)(wv[k4] >> (8 * (b - b0)));
+        }
+    }
+}
+
+// Persistent CTAs walk work items round-robin; one thread streams each item's
+// tiles (one contiguous, 512-byte aligned span of the blocked buffer) into a
+// stage with a 1-D bulk copy completed on an mbarrier, two stages deep.  Per
+// item:
+//  1. Thread (j = lane, q = warp) reads line j of its quads of tiles (a warp
+//     reads one 512-byte tile per instruction); word a of line j of tile cb
+//     holds row j + 32a, columns 4cb .. 4cb+3, so a 4x4 word transpose gives
+//     16 bytes of each of rows j, j+32, j+64, j+96, written to one of two
+//     shared row blocks.
+//  2. One barrier: the stage is free (thread 0 refills it) and the other row
+//     block is no longer read.
+//  3. Output chunks, each shifted into place from the 32-byte window around
+//     it.  Per-row mode: a warp writes 4 rows at a time, lane l taking chunk
+//     l % 8 of row l / 8 (one 128-bit store covers four contiguous runs), a
+//     9th chunk by the row's first lane.  Flat mode (rows back to back in
+//     memory, at most 128 columns): the item's rows are one contiguous span
+//     and threads take its chunks in order.
+template <bool kDimM>
+__global__ void __launch_bounds__(kThreads, 3)
+unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, const int32_t *__restrict__ ends,
+                   uint8_t *__restrict__ scales, int64_t row_stride, Shape s, int flat) {
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t *stages = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 127) & ~uintptr_t(127));
+    uint8_t *rowblks = stages + kInvStages * kInvStageBytes;
     __shared__ GroupTable table;
-    __shared__ __align__(16) uint8_t rowblk[kTileRows * kInvPitch];
+    __shared__ __align__(8) uint64_t full[kInvStages];
+    __shared__ InvItem items[kInvStages];
     const int tid = threadIdx.x;
     const int j = tid & 31;
     const int q = tid >> 5;
 
+    if (tid == 0) {
+#pragma unroll
+        for (int st = 0; st < kInvStages; ++st) mbar_init(&full[st], 1);
+        fence_mbar_init();
+    }
+    // L2 prefetch of the spans this CTA most likely reads first (item i at
+    // about 16 KB * i if every item were full); no observable value, so
+    // before the dependency wait.
+    if (tid == 32) {
+        for (int n = 0; n < kInvStages; ++n) {
+            const int64_t off = (int64_t)kTilesPerChunk * 512 * ((int)blockIdx.x + n * (int)gridDim.x);
+            if (off + kTilesPerChunk * 512 <= blocked_size) bulk_prefetch_l2(blocked + off, kTilesPerChunk * 512);
+        }
+    }
     grid_dependency_wait();
     if (q == 0) build_group_table<kDimM>(ends, s.G, kDimM ? s.rows : s.cols, s.col_chunks, table);
     __syncthreads();
+    grid_launch_dependents();
     const int total = total_items<kDimM>(table, s);
+    const int bid = blockIdx.x;
+    const int n_my = bid < total ? (total - 1 - bid) / (int)gridDim.x + 1 : 0;
 
-    for (int i = blockIdx.x; i < total; i += gridDim.x) {
-        const Item it = decode_item<kDimM>(table, s, i, 1);
-        uint4 w[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const int tile = 4 * q + t;
-            w[t] = tile < it.ntiles
-                       ? __ldg(reinterpret_cast<const uint4 *>(blocked + it.out_off + (int64_t)tile * 512 + 16 * j))
-                       : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-            *reinterpret_cast<uint4 *>(rowblk + (j + 32 * a) * kInvPitch + kInvLead + 16 * q) =
-                make_uint4(word_of(w[0], a), word_of(w[1], a), word_of(w[2], a), word_of(w[3], a));
-        __syncthreads();
+    auto decode = [&](int n) { return decode_inv<kDimM>(table, s, bid + n * (int)gridDim.x, scales, row_stride); };
+    auto issue = [&](const InvItem &it, int st) {
+        items[st] = it;
+        const uint32_t bytes = (uint32_t)it.nload * 512u;
+        mbar_arrive_expect_tx(&full[st], bytes);
+        bulk_load_g2s(stages + st * kInvStageBytes, blocked + it.src_off, bytes, &full[st]);
+    };
+    if (tid == 0)
+        for (int st = 0; st < kInvStages && st < n_my; ++st) issue(decode(st), st);
 
-        const int ncol = it.cols_valid;
-        const int npairs = it.rows_valid * kInvChunks;
-        for (int idx = tid; idx < npairs; idx += kThreads) {
-            const int r = idx / kInvChunks;
-            const int p = idx - r * kInvChunks;
-            uint8_t *row = scales + (int64_t)(it.y + r) * row_stride + it.x;   // item column 0 of row r
-            const int lead = (int)(reinterpret_cast<uintptr_t>(row) & 15u);
-            // global chunk p covers item columns [16p - lead, 16p - lead + 16)
-            const int c0 = 16 * p - lead;
-            if (c0 >= ncol) continue;
-            const uint8_t *win = rowblk + r * kInvPitch + 16 * p;           // shared bytes [16p, 16p + 32)
-            const uint4 lo = *reinterpret_cast<const uint4 *>(win);
-            const uint4 hi = *reinterpret_cast<const uint4 *>(win + 16);
-            const uint4 v = lead == 0 ? hi : realign(lo, hi, 16 - lead);
-            const int kmin = c0 < 0 ? -c0 : 0;
-            const int kmax = min(16, ncol - c0);
-            uint8_t *dst = row + c0;                                          // 16-byte aligned
-            if (kmin == 0 && kmax == 16) {
-                *reinterpret_cast<uint4 *>(dst) = v;
-            } else {
-                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    for (int n = 0; n < n_my; ++n) {
+        const int st = n % kInvStages;
+        // The refill of this stage is decoded while its current copy is in
+        // flight, so that only the copy itself is issued after the barrier.
+        const bool refill = tid == 0 && n + kInvStages < n_my;
+        InvItem next;
+        if (refill) next = decode(n + kInvStages);
+        const bool ok = mbar_wait_bounded(&full[st], (uint32_t)(n / kInvStages) & 1u);
+        InvItem it;
+        uint8_t *rowblk = rowblks + (n & 1) * kInvBlockBytes;
+        if (ok) {
+            it = items[st];
+            const uint8_t *stage = stages + st * kInvStageBytes;
+            const int nquads = (it.nload + 3) / 4;   // at most 9: warp 0 takes the ninth
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const int b0 = 4 * k4;
-                    if (b0 >= kmin && b0 + 4 <= kmax) {
-                        *reinterpret_cast<uint32_t *>(dst + b0) = wv[k4];
+            for (int pass = 0; pass < 2; ++pass) {
+                const int qq = q + 8 * pass;
+                if (qq >= nquads) break;
+                uint4 w[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const int tile = 4 * qq + t;
+                    w[t] = tile < it.nload ? *reinterpret_cast<const uint4 *>(stage + tile * 512 + 16 * j)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    const int r = j + 32 * a;
+                    if (!flat) {
+                        *reinterpret_cast<uint4 *>(rowblk + r * kInvPitch + 16 * qq) =
+                            make_uint4(word_of(w[0], a), word_of(w[1], a), word_of(w[2], a), word_of(w[3], a));
                     } else {
-                        for (int b = max(b0, kmin); b < min(b0 + 4, kmax); ++b)
-                            dst[b] = (uint8_t)(wv[k4] >> (8 * (b - b0)));
+                        // rows back to back: word-aligned (cols is a multiple of 4), stop at the row's end
+                        uint32_t *dst = reinterpret_cast<uint32_t *>(rowblk + r * s.cols) + 4 * qq;
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            if (16 * qq + 4 * t < s.cols) dst[t] = word_of(w[t], a);
                     }
                 }
             }
         }
-        __syncthreads();
+        if (__syncthreads_or(!ok)) {
+            // A copy never completed: flag it, wait (bounded) for the copies
+            // still in flight into this CTA's shared memory, and leave.
+            if (tid == 0) {
+                atomicOr(&g_inv_flags, kInvFlagWaitTimeout);
+                for (int m = n; m < n_my && m < n + kInvStages; ++m)
+                    mbar_wait_bounded(&full[m % kInvStages], (uint32_t)(m / kInvStages) & 1u);
+            }
+            return;
+        }
+        if (refill) issue(next, st);
+
+        if (!flat) {
+            uint8_t *base = scales + (int64_t)it.y * row_stride + it.x;   // item column 0 of row 0
+            const int p = j & 7;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int r = 4 * (q + 8 * k) + (j >> 3);
+                if (r < it.rows_valid) {
+                    uint8_t *row = base + (int64_t)r * row_stride;
+                    const int lead = (int)(reinterpret_cast<uintptr_t>(row) & 15u);
+                    // owned item columns: from the chunk boundary before column 0 (an item
+                    // that continues a run) and up to the next chunk boundary (unless last)
+                    const int lo_own = it.pre ? -lead : 0;
+                    const int hi_own = it.last ? it.ncol : kTilesPerChunk * 4 - lead;
+                    const uint8_t *src = rowblk + r * kInvPitch;
+                    const int c0 = 16 * p - lead;
+                    const int kmin = max(0, lo_own - c0), kmax = min(16, hi_own - c0);
+                    if (kmin < kmax) store16_part(row + c0, window16(src, c0 + it.pre, kInvPitch), kmin, kmax);
+                    // A ninth chunk exists only for the last item of a run whose
+                    // columns reach past the eighth chunk boundary; the row's first
+                    // lane writes it.  Kept out of the loop above so that the warp
+                    // does not issue a second pass for it.
+                    const int c8 = kTilesPerChunk * 4 - lead;
+                    if (p == 0 && c8 < hi_own)
+                        store16_part(row + c8, window16(src, c8 + it.pre, kInvPitch), 0, min(16, hi_own - c8));
+                }
+            }
+        } else {
+            const int span = it.rows_valid * s.cols;
+            uint8_t *base = scales + (int64_t)it.y * s.cols;   // the item's first byte
+            const int lead = (int)(reinterpret_cast<uintptr_t>(base) & 15u);
+            const int nch = (lead + span + 15) >> 4;
+            for (int p = tid; p < nch; p += kThreads) {
+                const int o = 16 * p - lead;
+                const int kmin = max(0, -o), kmax = min(16, span - o);
+                store16_part(base + o, window16(rowblk, o, kInvBlockBytes), kmin, kmax);
+            }
+        }
     }
 
     // Elements no group covers (rows past the last end for M, columns past
@@ -113,9 +300,9 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, const int32_t *__restric
     const int64_t zc0 = kDimM ? 0 : used;
     const int64_t zrows = s.rows - zr0, zcols = s.cols - zc0;
     if (zrows > 0 && zcols > 0) {
-        const int64_t n = zrows * zcols;
+        const int64_t nz = zrows * zcols;
         const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-        for (int64_t k = (int64_t)blockIdx.x * blockDim.x + tid; k < n; k += stride) {
+        for (int64_t k = (int64_t)blockIdx.x * blockDim.x + tid; k < nz; k += stride) {
             const int64_t r = zr0 + k / zcols, c = zc0 + k % zcols;
             scales[r * row_stride + c] = 0;
         }
@@ -136,11 +323,11 @@ __global__ void padded_starts_kernel(const int32_t *__restrict__ ends, int32_t *
 constexpr int64_t kMaxExtent = (1ll << 31) - (1ll << 14);
 
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, cudaStream_t stream, Args... args) {
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, int smem, cudaStream_t stream, Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -151,6 +338,36 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, cudaStream
 }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Per device, once: allow the inverse kernels their shared memory and note
+// how many CTAs of them fit on an SM.
+constexpr int kMaxDevices = 128;
+std::mutex g_inv_mu;
+int g_inv_grid[kMaxDevices];   // SMs x resident CTAs, 0 until set up
+
+cudaError_t inverse_grid_cap(int *cap) {
+    int dev = 0;
+    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_inv_mu);
+    if (g_inv_grid[dev] == 0) {
+        int sms = 0, occ_m = 0, occ_k = 0;
+        const cudaError_t steps[] = {
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev),
+            cudaFuncSetAttribute(unrearrange_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kInvSmemBytes),
+            cudaFuncSetAttribute(unrearrange_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kInvSmemBytes),
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_m, unrearrange_kernel<true>, kThreads, kInvSmemBytes),
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_k, unrearrange_kernel<false>, kThreads, kInvSmemBytes),
+        };
+        for (cudaError_t e : steps)
+            if (e != cudaSuccess) return e;
+        const int occ = occ_m < occ_k ? occ_m : occ_k;
+        if (occ < 1 || sms < 1) return cudaErrorInvalidConfiguration;
+        g_inv_grid[dev] = sms * occ;
+    }
+    *cap = g_inv_grid[dev];
+    return cudaSuccess;
+}
 
 Shape make_shape(int64_t rows, int64_t cols, int32_t G) {
     Shape s;
@@ -177,21 +394,32 @@ mx_status unrearrange(mx_group_dim dim, const uint8_t *blocked, int64_t rows, in
     const int64_t bound = dim_m ? (ceil_div(rows, 128) + G) * s.col_chunks
                                 : ceil_div(rows, 128) * (ceil_div(cols, kChunkCols) + G);
     if (bound > INT_MAX) return MX_ERR_UNSUPPORTED;
-    int dev = 0, sms = 0;
-    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return mx_record_cuda_error(e);
-    if (cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev); e != cudaSuccess)
-        return mx_record_cuda_error(e);
-    const int64_t cap = (int64_t)sms * 8 * 4;
+    int cap = 0;
+    if (cudaError_t e = inverse_grid_cap(&cap); e != cudaSuccess) return mx_record_cuda_error(e);
     const int grid = (int)(bound < 1 ? 1 : (bound < cap ? bound : cap));
-    cudaError_t e = dim_m ? launch_pdl(unrearrange_kernel<true>, grid, kThreads, stream, blocked, ends, scales,
-                                       row_stride, s)
-                          : launch_pdl(unrearrange_kernel<false>, grid, kThreads, stream, blocked, ends, scales,
-                                       row_stride, s);
+    const int64_t blocked_size = (int64_t)mx_rearranged_size(dim, rows, cols, G);
+    // flat mode: rows back to back, one item per row block, whole words
+    const int flat = dim_m && row_stride == cols && cols <= kTilesPerChunk * 4 && cols % 4 == 0 ? 1 : 0;
+    cudaError_t e = dim_m ? launch_pdl(unrearrange_kernel<true>, grid, kThreads, kInvSmemBytes, stream, blocked,
+                                       blocked_size, ends, scales, row_stride, s, flat)
+                          : launch_pdl(unrearrange_kernel<false>, grid, kThreads, kInvSmemBytes, stream, blocked,
+                                       blocked_size, ends, scales, row_stride, s, flat);
     return e == cudaSuccess ? MX_OK : mx_record_cuda_error(e);
 }
 
 }  // namespace
 }  // namespace mx
+
+// Read (and optionally clear) the inverse kernels' error flags; part of
+// mx_device_flags (C++ linkage, not part of the C ABI).
+cudaError_t mx_inverse_flags(unsigned int *flags, int clear) {
+    if (cudaError_t e = cudaMemcpyFromSymbol(flags, mx::g_inv_flags, sizeof(*flags)); e != cudaSuccess) return e;
+    if (clear) {
+        const unsigned int zero = 0;
+        if (cudaError_t e = cudaMemcpyToSymbol(mx::g_inv_flags, &zero, sizeof(zero)); e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
 
 extern "C" {
 
@@ -217,8 +445,9 @@ mx_status mx_padded_group_starts(mx_group_dim dim, int64_t rows, int64_t cols, c
     if (group_end_offsets == nullptr || starts == nullptr) return MX_ERR_INVALID_ARG;
     const mx::Shape s = mx::make_shape(rows, cols, num_groups);
     cudaError_t e = dim == MX_GROUPS_M
-                        ? mx::launch_pdl(mx::padded_starts_kernel<true>, 1, 32, stream, group_end_offsets, starts, s)
-                        : mx::launch_pdl(mx::padded_starts_kernel<false>, 1, 32, stream, group_end_offsets, starts, s);
+                        ? mx::launch_pdl(mx::padded_starts_kernel<true>, 1, 32, 0, stream, group_end_offsets, starts, s)
+                        : mx::launch_pdl(mx::padded_starts_kernel<false>, 1, 32, 0, stream, group_end_offsets, starts,
+                                         s);
     return e == cudaSuccess ? MX_OK : mx_record_cuda_error(e);
 }
 

@@ -835,6 +835,7 @@ mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t col
 
 // Shared with mx_inverse.cu (C++ linkage, not part of the C ABI).
 mx_status mx_record_cuda_error(cudaError_t e) { return mx::cuda_status(e); }
+cudaError_t mx_inverse_flags(unsigned int *flags, int clear);   // defined in mx_inverse.cu
 
 // ------------------------------------------------------------------ C ABI
 extern "C" {
@@ -884,10 +885,11 @@ const char *mx_status_string(mx_status status) {
 
 mx_status mx_device_flags(uint32_t *flags, int clear) {
     if (flags == nullptr) return MX_ERR_INVALID_ARG;
-    unsigned int v = 0;
+    unsigned int v = 0, inv = 0;
     if (cudaError_t e = cudaMemcpyFromSymbol(&v, mx::g_mx_flags, sizeof(v)); e != cudaSuccess)
         return mx::cuda_status(e);
-    *flags = v;
+    if (cudaError_t e = mx_inverse_flags(&inv, clear); e != cudaSuccess) return mx::cuda_status(e);
+    *flags = v | inv;
     if (clear) {
         const unsigned int zero = 0;
         if (cudaError_t e = cudaMemcpyToSymbol(mx::g_mx_flags, &zero, sizeof(zero)); e != cudaSuccess)
