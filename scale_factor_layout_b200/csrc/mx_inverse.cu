@@ -68,7 +68,11 @@ struct InvItem {
     int32_t nload;        // tiles loaded (own, plus the previous quad)
     int32_t pre;          // columns before the item's first one in the stage: 0 or 16
     int32_t last;         // 1 if the item ends its run
-    int32_t pad;
+    // Shift mode (row stride a multiple of 16, so every row of the item
+    // starts at the same offset within a 16-byte chunk):
+    int32_t lead;         // byte offset of item column 0 within its 16-byte chunk
+    int32_t nch;          // 16-byte output chunks per row the item owns a part of (<= 9)
+    int32_t partial;      // 1 if a row's first or last owned chunk is partial
 };
 
 // `out`, `row_stride`: the row-major output, to tell whether an item's first
@@ -104,7 +108,12 @@ __device__ __forceinline__ InvItem decode_inv(const GroupTable &t, const Shape &
     v.nload = it.ntiles + (pre ? kInvPreTiles : 0);
     v.src_off = it.out_off - (pre ? kInvPreTiles * 512 : 0);
     v.last = kTilesPerChunk * 4 * (k + 1) >= run ? 1 : 0;
-    v.pad = 0;
+    // owned columns [lo, hi) as in the store phase; chunk m covers item
+    // columns [16m - lead, 16m - lead + 16)
+    v.lead = (int)(reinterpret_cast<uintptr_t>(out + (int64_t)it.y * row_stride + it.x) & 15u);
+    const int hi = v.last ? v.ncol : kTilesPerChunk * 4 - v.lead;
+    v.nch = (hi + v.lead + 15) >> 4;
+    v.partial = ((!pre && v.lead != 0) || (v.last && ((v.ncol + v.lead) & 15) != 0)) ? 1 : 0;
     return v;
 }
 
@@ -138,27 +147,57 @@ __device__ __forceinline__ void store16_part(uint8_t *dst, const uint4 &v, int k
     }
 }
 
+// Bulk copy of one 16-byte chunk, shared -> global, writing only the bytes
+// whose bit is set in `mask` (bit i: byte i); both addresses 16-byte aligned.
+__device__ __forceinline__ void bulk_store16_masked(void *gdst, const void *ssrc, uint16_t mask) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.cp_mask [%0], [%1], 16, %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(gdst)), "r"(smem_addr(ssrc)), "h"(mask) : "memory");
+}
+
+// Shift mode: write output chunk p of a row whose chunks start at the
+// 16-byte aligned `row` and sit at `src` in shared memory; the item owns
+// bytes [lo, hi) of the row's chunk span.  Whole chunks are one 128-bit
+// store, partial ones one masked bulk copy.
+__device__ __forceinline__ void store_chunk_shift(uint8_t *row, const uint8_t *src, int p, int lo, int hi) {
+    const int kmin = max(0, lo - 16 * p), kmax = min(16, hi - 16 * p);
+    if (kmin >= kmax) return;
+    if (kmin == 0 && kmax == 16) {
+        *reinterpret_cast<uint4 *>(row + 16 * p) = *reinterpret_cast<const uint4 *>(src + 16 * p);
+    } else {
+        bulk_store16_masked(row + 16 * p, src + 16 * p, (uint16_t)(((1u << kmax) - 1u) & ~((1u << kmin) - 1u)));
+    }
+}
+
+constexpr int kModeRows = 0;    // rows start at different offsets within a 16-byte chunk
+constexpr int kModeShift = 1;   // row stride a multiple of 16: one offset for all rows of an item
+constexpr int kModeFlat = 2;    // rows back to back (stride == cols <= 128)
+
 // Persistent CTAs walk work items round-robin; one thread streams each item's
 // tiles (one contiguous, 512-byte aligned span of the blocked buffer) into a
-// stage with a 1-D bulk copy completed on an mbarrier, two stages deep.  Per
-// item:
-//  1. Thread (j = lane, q = warp) reads line j of its quads of tiles (a warp
-//     reads one 512-byte tile per instruction); word a of line j of tile cb
-//     holds row j + 32a, columns 4cb .. 4cb+3, so a 4x4 word transpose gives
-//     16 bytes of each of rows j, j+32, j+64, j+96, written to one of two
-//     shared row blocks.
+// stage with a 1-D bulk copy completed on an mbarrier, two stages deep.  Word
+// a of line j of tile cb holds row j + 32a, columns 4cb .. 4cb+3.  Per item:
+//  1. Transpose into one of two shared row blocks.  Thread (j = lane, q =
+//     warp) reads line j of a run of tiles (a warp reads one 512-byte tile
+//     per instruction), which gives rows j, j+32, j+64, j+96.
+//     Shift mode: row chunk m holds exactly the bytes of output chunk m (item
+//     columns from 16m - lead); five tile lines and a funnel shift give it,
+//     so the store phase moves aligned 16-byte chunks unchanged.  Other
+//     modes: quad qq of tiles gives columns 16qq .. 16qq+15 as loaded.
 //  2. One barrier: the stage is free (thread 0 refills it) and the other row
-//     block is no longer read.
-//  3. Output chunks, each shifted into place from the 32-byte window around
-//     it.  Per-row mode: a warp writes 4 rows at a time, lane l taking chunk
+//     block is no longer read (each thread first waits until its own bulk
+//     copies have read it).
+//  3. Output chunks.  A warp writes 4 rows at a time, lane l taking chunk
 //     l % 8 of row l / 8 (one 128-bit store covers four contiguous runs), a
-//     9th chunk by the row's first lane.  Flat mode (rows back to back in
-//     memory, at most 128 columns): the item's rows are one contiguous span
+//     ninth chunk by the row's first lane.  Shift mode: whole chunks are
+//     plain stores, partial ones (where a run starts or ends) masked bulk
+//     copies.  Rows mode: each chunk is shifted into place from the 32-byte
+//     window around it, partial ones stored by words and bytes.  Flat mode
+//     (rows back to back in memory): the item's rows are one contiguous span
 //     and threads take its chunks in order.
 template <bool kDimM>
 __global__ void __launch_bounds__(kThreads, 3)
 unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, const int32_t *__restrict__ ends,
-                   uint8_t *__restrict__ scales, int64_t row_stride, Shape s, int flat) {
+                   uint8_t *__restrict__ scales, int64_t row_stride, Shape s, int mode) {
     extern __shared__ uint8_t dyn_smem[];
     uint8_t *stages = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 127) & ~uintptr_t(127));
     uint8_t *rowblks = stages + kInvStages * kInvStageBytes;
@@ -168,6 +207,7 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
     const int tid = threadIdx.x;
     const int j = tid & 31;
     const int q = tid >> 5;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 
     if (tid == 0) {
 #pragma unroll
@@ -214,34 +254,66 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
         if (ok) {
             it = items[st];
             const uint8_t *stage = stages + st * kInvStageBytes;
-            const int nquads = (it.nload + 3) / 4;   // at most 9: warp 0 takes the ninth
+            if (mode == kModeShift) {
+                // Row chunk m: loaded columns from 16m + pre - lead, i.e. from
+                // byte sh / 8 of tile 4m + tb.
+                const int from = it.pre - it.lead;   // in [-15, 15]
+                const int tb = from >> 2;            // floor
+                const int sh = (from & 3) * 8;
 #pragma unroll
-            for (int pass = 0; pass < 2; ++pass) {
-                const int qq = q + 8 * pass;
-                if (qq >= nquads) break;
-                uint4 w[4];
+                for (int pass = 0; pass < 2; ++pass) {
+                    const int m = q + 8 * pass;      // at most 9 chunks: warp 0 takes the ninth
+                    if (m >= it.nch) break;
+                    uint4 w[5];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const int tile = 4 * qq + t;
-                    w[t] = tile < it.nload ? *reinterpret_cast<const uint4 *>(stage + tile * 512 + 16 * j)
-                                           : make_uint4(0u, 0u, 0u, 0u);
+                    for (int t = 0; t < 5; ++t) {
+                        const int tile = 4 * m + tb + t;
+                        w[t] = (tile >= 0 && tile < it.nload && (t < 4 || sh != 0))
+                                   ? *reinterpret_cast<const uint4 *>(stage + tile * 512 + 16 * j)
+                                   : zero;
+                    }
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        const uint32_t x0 = word_of(w[0], a), x1 = word_of(w[1], a), x2 = word_of(w[2], a),
+                                       x3 = word_of(w[3], a), x4 = word_of(w[4], a);
+                        *reinterpret_cast<uint4 *>(rowblk + (j + 32 * a) * kInvPitch + 16 * m) =
+                            make_uint4(funnel(x0, x1, sh), funnel(x1, x2, sh), funnel(x2, x3, sh), funnel(x3, x4, sh));
+                    }
                 }
+                // the masked bulk copies of the store phase read this row block
+                if (it.partial) fence_proxy_async_smem();
+            } else {
+                const int nquads = (it.nload + 3) / 4;   // at most 9: warp 0 takes the ninth
 #pragma unroll
-                for (int a = 0; a < 4; ++a) {
-                    const int r = j + 32 * a;
-                    if (!flat) {
-                        *reinterpret_cast<uint4 *>(rowblk + r * kInvPitch + 16 * qq) =
-                            make_uint4(word_of(w[0], a), word_of(w[1], a), word_of(w[2], a), word_of(w[3], a));
-                    } else {
-                        // rows back to back: word-aligned (cols is a multiple of 4), stop at the row's end
-                        uint32_t *dst = reinterpret_cast<uint32_t *>(rowblk + r * s.cols) + 4 * qq;
+                for (int pass = 0; pass < 2; ++pass) {
+                    const int qq = q + 8 * pass;
+                    if (qq >= nquads) break;
+                    uint4 w[4];
 #pragma unroll
-                        for (int t = 0; t < 4; ++t)
-                            if (16 * qq + 4 * t < s.cols) dst[t] = word_of(w[t], a);
+                    for (int t = 0; t < 4; ++t) {
+                        const int tile = 4 * qq + t;
+                        w[t] = tile < it.nload ? *reinterpret_cast<const uint4 *>(stage + tile * 512 + 16 * j) : zero;
+                    }
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        const int r = j + 32 * a;
+                        if (mode == kModeRows) {
+                            *reinterpret_cast<uint4 *>(rowblk + r * kInvPitch + 16 * qq) =
+                                make_uint4(word_of(w[0], a), word_of(w[1], a), word_of(w[2], a), word_of(w[3], a));
+                        } else {
+                            // rows back to back: word-aligned (cols is a multiple of 4), stop at the row's end
+                            uint32_t *dst = reinterpret_cast<uint32_t *>(rowblk + r * s.cols) + 4 * qq;
+#pragma unroll
+                            for (int t = 0; t < 4; ++t)
+                                if (16 * qq + 4 * t < s.cols) dst[t] = word_of(w[t], a);
+                        }
                     }
                 }
             }
         }
+        // this thread's masked copies of item n - 1 have read their row block,
+        // which item n + 1 overwrites after the barrier
+        bulk_wait_read<0>();
         if (__syncthreads_or(!ok)) {
             // A copy never completed: flag it, wait (bounded) for the copies
             // still in flight into this CTA's shared memory, and leave.
@@ -254,9 +326,26 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
         }
         if (refill) issue(next, st);
 
-        if (!flat) {
+        const int p = j & 7;
+        if (mode == kModeShift) {
+            // the 16-byte aligned start of row 0's first chunk; the item owns
+            // bytes [lo, hi) of each row's chunk span
+            uint8_t *base = scales + (int64_t)it.y * row_stride + it.x - it.lead;
+            const int lo = it.pre ? 0 : it.lead;
+            const int hi = (it.last ? it.ncol : kTilesPerChunk * 4 - it.lead) + it.lead;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int r = 4 * (q + 8 * k) + (j >> 3);
+                if (r < it.rows_valid) {
+                    uint8_t *row = base + (int64_t)r * row_stride;
+                    const uint8_t *src = rowblk + r * kInvPitch;
+                    store_chunk_shift(row, src, p, lo, hi);
+                    if (p == 0 && it.nch > 8) store_chunk_shift(row, src, 8, lo, hi);
+                }
+            }
+            if (it.partial) bulk_commit();
+        } else if (mode == kModeRows) {
             uint8_t *base = scales + (int64_t)it.y * row_stride + it.x;   // item column 0 of row 0
-            const int p = j & 7;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int r = 4 * (q + 8 * k) + (j >> 3);
@@ -273,7 +362,7 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
                     if (kmin < kmax) store16_part(row + c0, window16(src, c0 + it.pre, kInvPitch), kmin, kmax);
                     // A ninth chunk exists only for the last item of a run whose
                     // columns reach past the eighth chunk boundary; the row's first
-                    // lane writes it.  Kept out of the loop above so that the warp
+                    // lane writes it.  Kept out of the store above so that the warp
                     // does not issue a second pass for it.
                     const int c8 = kTilesPerChunk * 4 - lead;
                     if (p == 0 && c8 < hi_own)
@@ -285,13 +374,15 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
             uint8_t *base = scales + (int64_t)it.y * s.cols;   // the item's first byte
             const int lead = (int)(reinterpret_cast<uintptr_t>(base) & 15u);
             const int nch = (lead + span + 15) >> 4;
-            for (int p = tid; p < nch; p += kThreads) {
-                const int o = 16 * p - lead;
+            for (int c = tid; c < nch; c += kThreads) {
+                const int o = 16 * c - lead;
                 const int kmin = max(0, -o), kmax = min(16, span - o);
                 store16_part(base + o, window16(rowblk, o, kInvBlockBytes), kmin, kmax);
             }
         }
     }
+    // the masked copies read shared memory, which must outlive them
+    bulk_wait_all();
 
     // Elements no group covers (rows past the last end for M, columns past
     // it for K) are written as zeros; the gaps between rows are not touched.
@@ -399,11 +490,13 @@ mx_status unrearrange(mx_group_dim dim, const uint8_t *blocked, int64_t rows, in
     const int grid = (int)(bound < 1 ? 1 : (bound < cap ? bound : cap));
     const int64_t blocked_size = (int64_t)mx_rearranged_size(dim, rows, cols, G);
     // flat mode: rows back to back, one item per row block, whole words
-    const int flat = dim_m && row_stride == cols && cols <= kTilesPerChunk * 4 && cols % 4 == 0 ? 1 : 0;
+    const int mode = dim_m && row_stride == cols && cols <= kTilesPerChunk * 4 && cols % 4 == 0 ? kModeFlat
+                     : (row_stride & 15) == 0                                                  ? kModeShift
+                                                                                                : kModeRows;
     cudaError_t e = dim_m ? launch_pdl(unrearrange_kernel<true>, grid, kThreads, kInvSmemBytes, stream, blocked,
-                                       blocked_size, ends, scales, row_stride, s, flat)
+                                       blocked_size, ends, scales, row_stride, s, mode)
                           : launch_pdl(unrearrange_kernel<false>, grid, kThreads, kInvSmemBytes, stream, blocked,
-                                       blocked_size, ends, scales, row_stride, s, flat);
+                                       blocked_size, ends, scales, row_stride, s, mode);
     return e == cudaSuccess ? MX_OK : mx_record_cuda_error(e);
 }
 

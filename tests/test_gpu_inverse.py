@@ -51,6 +51,23 @@ def test_inverse_strided_misaligned_out(mxlib, orc, name, pad, misalign):
     _inverse_check(synth.NAMED[name](), orc, out_pad=pad, misalign=misalign)
 
 
+@pytest.mark.parametrize("misalign", range(16))
+def test_inverse_every_chunk_offset(mxlib, orc, misalign):
+    """Row strides that are multiples of 16 with the output base at every
+    offset within a 16-byte chunk: each row of an item then starts at the same
+    offset, and every head and tail mask of a partial chunk occurs (K groups
+    start at arbitrary columns; M rows wider than one 128-column item)."""
+    rng = np.random.default_rng(4100 + misalign)
+    rows, cols = 300, 700
+    scales = rng.integers(1, 255, size=(rows, cols), dtype=np.uint8)
+    cuts = np.sort(rng.choice(np.arange(1, cols), size=7, replace=False))
+    k_case = synth.Case("shiftK", synth.DIM_K, scales, np.append(cuts, cols).astype(np.int32), 0)
+    _inverse_check(k_case, orc, out_pad=(-cols) % 16 + 16, misalign=misalign)
+    m_scales = rng.integers(1, 255, size=(rows, 150), dtype=np.uint8)
+    m_case = synth.Case("shiftM", synth.DIM_M, m_scales, np.array([0, 77, 200, 200, 300], np.int32), 0)
+    _inverse_check(m_case, orc, out_pad=(-150) % 16, misalign=misalign)
+
+
 def test_inverse_sweep_subset(mxlib, orc):
     for i_rows in range(len(synth.SWEEP_ROWS)):
         for i_k in (0, 3, 6):
