@@ -62,6 +62,7 @@ __device__ unsigned int g_inv_flags = 0;
 // run starts or ends.
 struct InvItem {
     int64_t src_off;      // blocked offset of the first tile loaded
+    int64_t src2_off;     // merged seam: blocked offset of the previous group's tiles
     int32_t x, y;         // first output column and row of the item
     int32_t rows_valid;   // rows with data
     int32_t ncol;         // item columns with data (<= 128)
@@ -71,9 +72,24 @@ struct InvItem {
     // Shift mode (row stride a multiple of 16, so every row of the item
     // starts at the same offset within a 16-byte chunk):
     int32_t lead;         // byte offset of item column 0 within its 16-byte chunk
+    int32_t lo, hi;       // owned bytes [lo, hi) of a row, counted from its first chunk
     int32_t nch;          // 16-byte output chunks per row the item owns a part of (<= 9)
     int32_t partial;      // 1 if a row's first or last owned chunk is partial
+    int32_t merge;        // 1 if the item writes the seam chunk before its group whole
+    int32_t n2;           // merged seam: tiles of the previous group loaded (<= 4)
+    int32_t b0;           // merged seam: byte of the first needed column in the first of them
+    int32_t pad;
 };
+
+// Groups along K, shift mode: a 16-byte output chunk that holds the seam
+// between a group and the next non-empty one (the seam `ls` bytes into the
+// chunk, ls != 0) is written whole by the later group's first item when the
+// earlier group has the ls columns before the seam within 4 of its tiles and
+// the later group fills the rest of the chunk; otherwise both items write
+// their part of it (masked).  Both items evaluate this same function.
+__device__ __forceinline__ bool seam_whole(int w_prev, int w_next, int ls) {
+    return ls != 0 && w_prev >= ls && ((w_prev - ls) & 3) + ls <= 16 && w_next >= 16 - ls;
+}
 
 // `out`, `row_stride`: the row-major output, to tell whether an item's first
 // column can start mid-chunk (only then is the quad before it needed).
@@ -81,23 +97,24 @@ template <bool kDimM>
 __device__ __forceinline__ InvItem decode_inv(const GroupTable &t, const Shape &s, int i, const uint8_t *out,
                                               int64_t row_stride) {
     const Item it = decode_item<kDimM>(t, s, i, 1);
-    int k, run;   // item's chunk index in its run, and the run's column count
+    int k, run, g, rb = 0;   // item's chunk index in its run, the run's column count, group, row band
     if (kDimM) {
-        const int g = find_group(t, s.G, i);
+        g = find_group(t, s.G, i);
         const int local = i - t.istart[g];
         k = local - (local / s.col_chunks) * s.col_chunks;
         run = s.cols;
     } else {
         const int per_band = t.istart[kMaxGroups];
-        const int local = i - (i / per_band) * per_band;
-        const int g = find_group(t, s.G, local);
+        rb = i / per_band;
+        const int local = i - rb * per_band;
+        g = find_group(t, s.G, local);
         k = local - t.istart[g];
         run = t.size[g];
     }
     // every row of the item starts 16-byte aligned: no chunk straddles the
     // item's first column, so nothing before it is needed
-    const bool aligned = (row_stride & 15) == 0 &&
-                         ((reinterpret_cast<uintptr_t>(out + (int64_t)it.y * row_stride + it.x) & 15u) == 0);
+    const bool shift = (row_stride & 15) == 0;
+    const bool aligned = shift && ((reinterpret_cast<uintptr_t>(out + (int64_t)it.y * row_stride + it.x) & 15u) == 0);
     const bool pre = k > 0 && !aligned;
     InvItem v;
     v.x = it.x;
@@ -108,12 +125,40 @@ __device__ __forceinline__ InvItem decode_inv(const GroupTable &t, const Shape &
     v.nload = it.ntiles + (pre ? kInvPreTiles : 0);
     v.src_off = it.out_off - (pre ? kInvPreTiles * 512 : 0);
     v.last = kTilesPerChunk * 4 * (k + 1) >= run ? 1 : 0;
-    // owned columns [lo, hi) as in the store phase; chunk m covers item
-    // columns [16m - lead, 16m - lead + 16)
+    // owned columns as in the store phase; chunk m covers item columns
+    // [16m - lead, 16m - lead + 16)
     v.lead = (int)(reinterpret_cast<uintptr_t>(out + (int64_t)it.y * row_stride + it.x) & 15u);
-    const int hi = v.last ? v.ncol : kTilesPerChunk * 4 - v.lead;
-    v.nch = (hi + v.lead + 15) >> 4;
-    v.partial = ((!pre && v.lead != 0) || (v.last && ((v.ncol + v.lead) & 15) != 0)) ? 1 : 0;
+    v.lo = pre ? 0 : v.lead;
+    int hi_c = v.last ? v.ncol : kTilesPerChunk * 4 - v.lead;
+    v.merge = 0;
+    v.n2 = 0;
+    v.b0 = 0;
+    v.src2_off = 0;
+    v.pad = 0;
+    if (!kDimM && shift) {
+        if (k == 0 && v.lead != 0) {
+            int gp = g - 1;
+            while (gp >= 0 && t.size[gp] == 0) --gp;
+            if (gp >= 0 && seam_whole(t.size[gp], t.size[g], v.lead)) {
+                const int wp = t.size[gp], Wp = t.pstart[gp + 1] - t.pstart[gp];
+                const int t0 = (wp - v.lead) >> 2;
+                v.merge = 1;
+                v.lo = 0;
+                v.n2 = min(kInvPreTiles, Wp / 4 - t0);
+                v.b0 = (wp - v.lead) & 3;
+                v.src2_off = (int64_t)s.padded_rows * t.pstart[gp] + (int64_t)rb * kTileRows * Wp + 512ll * t0;
+            }
+        }
+        if (v.last) {
+            const int ls = (v.lead + v.ncol) & 15;
+            int gn = g + 1;
+            while (gn < s.G && t.size[gn] == 0) ++gn;
+            if (gn < s.G && seam_whole(t.size[g], t.size[gn], ls)) hi_c = v.ncol - ls;
+        }
+    }
+    v.hi = hi_c + v.lead;
+    v.nch = (v.hi + 15) >> 4;
+    v.partial = ((v.lo & 15) != 0 || (v.hi & 15) != 0) ? 1 : 0;
     return v;
 }
 
@@ -234,9 +279,12 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
     auto decode = [&](int n) { return decode_inv<kDimM>(table, s, bid + n * (int)gridDim.x, scales, row_stride); };
     auto issue = [&](const InvItem &it, int st) {
         items[st] = it;
-        const uint32_t bytes = (uint32_t)it.nload * 512u;
-        mbar_arrive_expect_tx(&full[st], bytes);
+        const uint32_t bytes = (uint32_t)it.nload * 512u, bytes2 = (uint32_t)it.n2 * 512u;
+        mbar_arrive_expect_tx(&full[st], bytes + bytes2);
         bulk_load_g2s(stages + st * kInvStageBytes, blocked + it.src_off, bytes, &full[st]);
+        // a merged seam's tiles of the previous group, after the item's own (at most 32: no quad before)
+        if (bytes2) bulk_load_g2s(stages + st * kInvStageBytes + kTilesPerChunk * 512, blocked + it.src2_off, bytes2,
+                                  &full[st]);
     };
     if (tid == 0)
         for (int st = 0; st < kInvStages && st < n_my; ++st) issue(decode(st), st);
@@ -278,6 +326,33 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
                                        x3 = word_of(w[3], a), x4 = word_of(w[4], a);
                         *reinterpret_cast<uint4 *>(rowblk + (j + 32 * a) * kInvPitch + 16 * m) =
                             make_uint4(funnel(x0, x1, sh), funnel(x1, x2, sh), funnel(x2, x3, sh), funnel(x3, x4, sh));
+                    }
+                    if (!kDimM && m == 0 && it.merge) {
+                        // Seam chunk: bytes [0, lead) are the previous group's last
+                        // columns, from its tiles after the item's own in the stage;
+                        // this thread just wrote the chunk's other bytes.
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            w[t] = t < it.n2 ? *reinterpret_cast<const uint4 *>(stage + (kTilesPerChunk + t) * 512 + 16 * j)
+                                             : zero;
+                        const int sh0 = it.b0 * 8;
+                        uint32_t keep[4];   // per word, the bytes below lead
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int nb = min(max(it.lead - 4 * e, 0), 4);
+                            keep[e] = nb == 4 ? 0xffffffffu : (1u << (8 * nb)) - 1u;
+                        }
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) {
+                            const uint32_t p0 = word_of(w[0], a), p1 = word_of(w[1], a), p2 = word_of(w[2], a),
+                                           p3 = word_of(w[3], a);
+                            uint4 *dst = reinterpret_cast<uint4 *>(rowblk + (j + 32 * a) * kInvPitch);
+                            const uint4 own = *dst;
+                            *dst = make_uint4((funnel(p0, p1, sh0) & keep[0]) | (own.x & ~keep[0]),
+                                              (funnel(p1, p2, sh0) & keep[1]) | (own.y & ~keep[1]),
+                                              (funnel(p2, p3, sh0) & keep[2]) | (own.z & ~keep[2]),
+                                              (funnel(p3, 0u, sh0) & keep[3]) | (own.w & ~keep[3]));
+                        }
                     }
                 }
                 // the masked bulk copies of the store phase read this row block
@@ -331,8 +406,7 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
             // the 16-byte aligned start of row 0's first chunk; the item owns
             // bytes [lo, hi) of each row's chunk span
             uint8_t *base = scales + (int64_t)it.y * row_stride + it.x - it.lead;
-            const int lo = it.pre ? 0 : it.lead;
-            const int hi = (it.last ? it.ncol : kTilesPerChunk * 4 - it.lead) + it.lead;
+            const int lo = it.lo, hi = it.hi;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int r = 4 * (q + 8 * k) + (j >> 3);
