@@ -367,10 +367,16 @@ rearrange_tma_k(const __grid_constant__ CUtensorMap tmap, const int32_t *__restr
 // read zeros).  Rows sit at pitch row_stride in shared memory; with the
 // stride a multiple of 4 every row starts on a word, and the transpose reads
 // 32-bit words.  Pipeline, staging and bulk stores follow rearrange_tma_m.
+//
+// Two instances: 8 warps and 4 stages for rows of more than 64 padded
+// columns; 4 warps and 2 stages for rows of at most 64 (one quad of tiles
+// per warp), small enough per CTA that about one row block per CTA is
+// resident at once on a B200 (1032 row blocks of a 131072-row input).
 constexpr int kFlatBoxWords = 256;
 constexpr int kFlatBoxBytes = kFlatBoxWords * 4;
 constexpr int kFlatStages = 4;
 constexpr int kFlatMaxStride = 256;
+constexpr int kFlatNarrowCols = 64;   // padded columns up to which the 4-warp instance runs
 
 struct FlatShape {
     int32_t row_stride;     // bytes, a multiple of 4
@@ -378,16 +384,19 @@ struct FlatShape {
     int32_t staging_bytes;  // tiles per row block * 512, rounded to 1 KB
 };
 
-__global__ void __launch_bounds__(kThreads)
+template <int kWarpsF, int kStagesF>
+__global__ void __launch_bounds__(kWarpsF * 32)
 rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restrict__ ends,
                    uint8_t *__restrict__ out, int64_t out_size, Shape s, FlatShape f) {
+    static_assert(kWarpsF == 8 || kWarpsF == 4, "8 warps (up to 16 quads of tiles) or 4 (up to 4)");
+    constexpr int kPasses = kWarpsF == 8 ? 2 : 1;   // quads of tiles per thread
     extern __shared__ uint8_t dyn_smem[];
     uint8_t *stages = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(dyn_smem) + 127) & ~uintptr_t(127));
-    uint8_t *staging = stages + kFlatStages * f.stage_bytes;
+    uint8_t *staging = stages + kStagesF * f.stage_bytes;
     __shared__ GroupTable table;
-    __shared__ __align__(8) uint64_t full[kFlatStages];
-    __shared__ Item items[kFlatStages];
+    __shared__ __align__(8) uint64_t full[kStagesF];
+    __shared__ Item items[kStagesF];
 
     const int tid = threadIdx.x;
     const int j = tid & 31;
@@ -399,13 +408,13 @@ rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__re
     if (tid == 0) {
         tma_prefetch_desc(&tmap);
 #pragma unroll
-        for (int st = 0; st < kFlatStages; ++st) mbar_init(&full[st], 1);
+        for (int st = 0; st < kStagesF; ++st) mbar_init(&full[st], 1);
         fence_mbar_init();
     }
     // L2 prefetch of the row blocks this CTA most likely takes first (row
     // block i if no group were padded); no observable value, so before the wait.
     if (tid == 32) {
-        for (int n = 0; n < kFlatStages; ++n) {
+        for (int n = 0; n < kStagesF; ++n) {
             const int64_t y = (int64_t)kTileRows * ((int)blockIdx.x + n * (int)gridDim.x);
             if (y >= s.rows) break;
             const int64_t w0 = ((y * L) >> 4) << 2;
@@ -444,22 +453,22 @@ rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__re
     };
 
     if (tid == 0)
-        for (int st = 0; st < kFlatStages && st < n_my; ++st) issue(st, st);
+        for (int st = 0; st < kStagesF && st < n_my; ++st) issue(st, st);
 
     int64_t prev_off = 0;
     uint32_t prev_bytes = 0;
     for (int n = 0; n < n_my; ++n) {
-        const int st = n % kFlatStages;
-        const uint32_t parity = (uint32_t)(n / kFlatStages) & 1u;
+        const int st = n % kStagesF;
+        const uint32_t parity = (uint32_t)(n / kStagesF) & 1u;
         const bool ok = mbar_wait_bounded(&full[st], parity);
         Item it;
-        uint32_t wv[2][4][4];   // [quad pass][row a][word t]
+        uint32_t wv[kPasses][4][4];   // [quad pass][row a][word t]
         if (ok) {
             it = items[st];
             const uint8_t *stage = stages + st * f.stage_bytes + it.delta;
 #pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                const int qq = q + 8 * p;
+            for (int p = 0; p < kPasses; ++p) {
+                const int qq = q + kWarpsF * p;
 #pragma unroll
                 for (int a = 0; a < 4; ++a) {
                     const uint32_t *row = reinterpret_cast<const uint32_t *>(stage + (j + 32 * a) * L) + 4 * qq;
@@ -472,8 +481,8 @@ rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__re
         if (__syncthreads_or(!ok)) {
             if (tid == 0) {
                 atomicOr(&g_mx_flags, kFlagWaitTimeout);
-                for (int m = n; m < n_my && m < n + kFlatStages; ++m)
-                    mbar_wait_bounded(&full[m % kFlatStages], (uint32_t)(m / kFlatStages) & 1u);
+                for (int m = n; m < n_my && m < n + kStagesF; ++m)
+                    mbar_wait_bounded(&full[m % kStagesF], (uint32_t)(m / kStagesF) & 1u);
             }
             return;
         }
@@ -484,12 +493,12 @@ rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__re
             }
             prev_off = it.out_off;
             prev_bytes = (uint32_t)it.ntiles * 512u;
-            if (n + kFlatStages < n_my) issue(n + kFlatStages, st);
+            if (n + kStagesF < n_my) issue(n + kStagesF, st);
         }
         uint8_t *stg = staging + (n & 1) * f.staging_bytes;
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const int qq = q + 8 * p;
+        for (int p = 0; p < kPasses; ++p) {
+            const int qq = q + kWarpsF * p;
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
                 const int tile = 4 * qq + t;
@@ -629,7 +638,10 @@ FlatShape flat_shape(int64_t row_stride, int64_t padded_cols) {
     return f;
 }
 
-int flat_smem_bytes(const FlatShape &f) { return kFlatStages * f.stage_bytes + 2 * f.staging_bytes + 128; }
+int flat_smem_bytes(const FlatShape &f, int stages) { return stages * f.stage_bytes + 2 * f.staging_bytes + 128; }
+
+// The flat kernel instance for rows of `padded_cols` columns.
+bool flat_narrow(int64_t padded_cols) { return padded_cols <= kFlatNarrowCols; }
 
 // The CUDA error behind the calling thread's latest MX_ERR_CUDA.
 thread_local cudaError_t t_last_error = cudaSuccess;
@@ -673,9 +685,13 @@ mx_status device_info(const DeviceInfo **out) {
     if (!d.ready) {
         if (cudaError_t e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev); e != cudaSuccess)
             return cuda_status(e);
-        const int flat_max = flat_smem_bytes(flat_shape(kFlatMaxStride, kFlatMaxStride));
+        const int flat_max = flat_smem_bytes(flat_shape(kFlatMaxStride, kFlatMaxStride), kFlatStages);
+        const int flat_narrow_max = flat_smem_bytes(flat_shape(kFlatMaxStride, kFlatNarrowCols), 2);
         const cudaError_t setup[] = {
-            cudaFuncSetAttribute(rearrange_flat_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, flat_max),
+            cudaFuncSetAttribute(rearrange_flat_tma<8, kFlatStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 flat_max),
+            cudaFuncSetAttribute(rearrange_flat_tma<4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 flat_narrow_max),
             cudaFuncSetAttribute(rearrange_tma_m, cudaFuncAttributeMaxDynamicSharedMemorySize, tma_smem_bytes<true>()),
             cudaFuncSetAttribute(rearrange_tma_k, cudaFuncAttributeMaxDynamicSharedMemorySize, tma_smem_bytes<false>()),
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_tma[1], rearrange_tma_m, kThreads,
@@ -697,10 +713,11 @@ mx_status device_info(const DeviceInfo **out) {
 // while the previous kernel in the stream drains; it waits for that kernel's
 // completion (griddepcontrol.wait) before touching global memory.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int smem, cudaStream_t stream, Args... args) {
+cudaError_t launch_pdl_block(void (*kernel)(KArgs...), int grid, int block, int smem, cudaStream_t stream,
+                             Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -709,6 +726,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int smem, cudaStream_
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int smem, cudaStream_t stream, Args... args) {
+    return launch_pdl_block(kernel, grid, kThreads, smem, stream, args...);
 }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -812,14 +834,17 @@ mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t col
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cuda_status(static_cast<cudaError_t>(r));   // driver code
         const FlatShape f = flat_shape(row_stride, s.padded_cols);
-        const int smem = flat_smem_bytes(f);
+        const bool narrow = flat_narrow(s.padded_cols);
+        auto kernel = narrow ? rearrange_flat_tma<4, 2> : rearrange_flat_tma<8, kFlatStages>;
+        const int block = narrow ? 128 : kThreads;
+        const int smem = flat_smem_bytes(f, narrow ? 2 : kFlatStages);
         int occ = 0;
-        if (cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rearrange_flat_tma, kThreads, smem);
+        if (cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, block, smem);
             e != cudaSuccess || occ < 1)
             return cuda_status(e != cudaSuccess ? e : cudaErrorInvalidConfiguration);
         const int64_t cap = (int64_t)d->sms * occ;
         const int grid = (int)(work < cap ? work : cap);
-        launched = launch_pdl(rearrange_flat_tma, grid, smem, stream, map, ends, out, (int64_t)size, s, f);
+        launched = launch_pdl_block(kernel, grid, block, smem, stream, map, ends, out, (int64_t)size, s, f);
     } else {
         const int64_t cap = (int64_t)d->sms * d->occ_fallback * 4;
         const int grid = (int)(work < cap ? work : cap);
