@@ -49,6 +49,13 @@ constexpr int kInvStages = 2;                                           // items
 constexpr int kInvStageBytes = (kTilesPerChunk + kInvPreTiles) * 512;   // 18 KB
 constexpr int kInvBlockBytes = kTileRows * kInvPitch;                   // 18 KB
 constexpr int kInvSmemBytes = kInvStages * kInvStageBytes + 2 * kInvBlockBytes + 128;
+// The narrow instance (4 warps) runs flat mode for rows of at most 64 padded
+// columns: an item is at most 16 tiles, its rows at most 8 KB together, so a
+// CTA is small enough that about one row block per CTA is resident at once.
+constexpr int kInvNarrowCols = 64;
+constexpr int kInvNarrowStageBytes = (kInvNarrowCols / 4) * 512;             // 8 KB
+constexpr int kInvNarrowBlockBytes = kTileRows * kInvNarrowCols;             // 8 KB
+constexpr int kInvNarrowSmemBytes = kInvStages * kInvNarrowStageBytes + 2 * kInvNarrowBlockBytes + 128;
 constexpr uint32_t kInvFlagWaitTimeout = 1u;
 
 // Error flags of the inverse kernels (a pipeline wait ran past its limit).
@@ -239,13 +246,19 @@ constexpr int kModeFlat = 2;    // rows back to back (stride == cols <= 128)
 //     window around it, partial ones stored by words and bytes.  Flat mode
 //     (rows back to back in memory): the item's rows are one contiguous span
 //     and threads take its chunks in order.
-template <bool kDimM>
-__global__ void __launch_bounds__(kThreads, 3)
+template <bool kDimM, int kWarpsI>
+__global__ void __launch_bounds__(kWarpsI * 32, kWarpsI == 8 ? 3 : 6)
 unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, const int32_t *__restrict__ ends,
                    uint8_t *__restrict__ scales, int64_t row_stride, Shape s, int mode) {
+    static_assert(kWarpsI == 8 || kWarpsI == 4, "8 warps (every mode) or 4 (narrow flat rows)");
+    constexpr bool kNarrow = kWarpsI == 4;
+    constexpr int kThr = kWarpsI * 32;
+    constexpr int kStageB = kNarrow ? kInvNarrowStageBytes : kInvStageBytes;
+    constexpr int kBlockB = kNarrow ? kInvNarrowBlockBytes : kInvBlockBytes;
+    constexpr int kPasses = kNarrow ? 1 : 2;   // quads of tiles per thread (at most 4, or 9)
     extern __shared__ uint8_t dyn_smem[];
     uint8_t *stages = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 127) & ~uintptr_t(127));
-    uint8_t *rowblks = stages + kInvStages * kInvStageBytes;
+    uint8_t *rowblks = stages + kInvStages * kStageB;
     __shared__ GroupTable table;
     __shared__ __align__(8) uint64_t full[kInvStages];
     __shared__ InvItem items[kInvStages];
@@ -264,8 +277,9 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
     // before the dependency wait.
     if (tid == 32) {
         for (int n = 0; n < kInvStages; ++n) {
-            const int64_t off = (int64_t)kTilesPerChunk * 512 * ((int)blockIdx.x + n * (int)gridDim.x);
-            if (off + kTilesPerChunk * 512 <= blocked_size) bulk_prefetch_l2(blocked + off, kTilesPerChunk * 512);
+            constexpr int kSpan = kNarrow ? kStageB : kTilesPerChunk * 512;
+            const int64_t off = (int64_t)kSpan * ((int)blockIdx.x + n * (int)gridDim.x);
+            if (off + kSpan <= blocked_size) bulk_prefetch_l2(blocked + off, kSpan);
         }
     }
     grid_dependency_wait();
@@ -281,9 +295,9 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
         items[st] = it;
         const uint32_t bytes = (uint32_t)it.nload * 512u, bytes2 = (uint32_t)it.n2 * 512u;
         mbar_arrive_expect_tx(&full[st], bytes + bytes2);
-        bulk_load_g2s(stages + st * kInvStageBytes, blocked + it.src_off, bytes, &full[st]);
+        bulk_load_g2s(stages + st * kStageB, blocked + it.src_off, bytes, &full[st]);
         // a merged seam's tiles of the previous group, after the item's own (at most 32: no quad before)
-        if (bytes2) bulk_load_g2s(stages + st * kInvStageBytes + kTilesPerChunk * 512, blocked + it.src2_off, bytes2,
+        if (bytes2) bulk_load_g2s(stages + st * kStageB + kTilesPerChunk * 512, blocked + it.src2_off, bytes2,
                                   &full[st]);
     };
     if (tid == 0)
@@ -298,11 +312,11 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
         if (refill) next = decode(n + kInvStages);
         const bool ok = mbar_wait_bounded(&full[st], (uint32_t)(n / kInvStages) & 1u);
         InvItem it;
-        uint8_t *rowblk = rowblks + (n & 1) * kInvBlockBytes;
+        uint8_t *rowblk = rowblks + (n & 1) * kBlockB;
         if (ok) {
             it = items[st];
-            const uint8_t *stage = stages + st * kInvStageBytes;
-            if (mode == kModeShift) {
+            const uint8_t *stage = stages + st * kStageB;
+            if (!kNarrow && mode == kModeShift) {
                 // Row chunk m: loaded columns from 16m + pre - lead, i.e. from
                 // byte sh / 8 of tile 4m + tb.
                 const int from = it.pre - it.lead;   // in [-15, 15]
@@ -360,8 +374,8 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
             } else {
                 const int nquads = (it.nload + 3) / 4;   // at most 9: warp 0 takes the ninth
 #pragma unroll
-                for (int pass = 0; pass < 2; ++pass) {
-                    const int qq = q + 8 * pass;
+                for (int pass = 0; pass < kPasses; ++pass) {
+                    const int qq = q + kWarpsI * pass;
                     if (qq >= nquads) break;
                     uint4 w[4];
 #pragma unroll
@@ -372,7 +386,7 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
 #pragma unroll
                     for (int a = 0; a < 4; ++a) {
                         const int r = j + 32 * a;
-                        if (mode == kModeRows) {
+                        if (!kNarrow && mode == kModeRows) {
                             *reinterpret_cast<uint4 *>(rowblk + r * kInvPitch + 16 * qq) =
                                 make_uint4(word_of(w[0], a), word_of(w[1], a), word_of(w[2], a), word_of(w[3], a));
                         } else {
@@ -402,7 +416,7 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
         if (refill) issue(next, st);
 
         const int p = j & 7;
-        if (mode == kModeShift) {
+        if (!kNarrow && mode == kModeShift) {
             // the 16-byte aligned start of row 0's first chunk; the item owns
             // bytes [lo, hi) of each row's chunk span
             uint8_t *base = scales + (int64_t)it.y * row_stride + it.x - it.lead;
@@ -418,7 +432,7 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
                 }
             }
             if (it.partial) bulk_commit();
-        } else if (mode == kModeRows) {
+        } else if (!kNarrow && mode == kModeRows) {
             uint8_t *base = scales + (int64_t)it.y * row_stride + it.x;   // item column 0 of row 0
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -448,10 +462,10 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
             uint8_t *base = scales + (int64_t)it.y * s.cols;   // the item's first byte
             const int lead = (int)(reinterpret_cast<uintptr_t>(base) & 15u);
             const int nch = (lead + span + 15) >> 4;
-            for (int c = tid; c < nch; c += kThreads) {
+            for (int c = tid; c < nch; c += kThr) {
                 const int o = 16 * c - lead;
                 const int kmin = max(0, -o), kmax = min(16, span - o);
-                store16_part(base + o, window16(rowblk, o, kInvBlockBytes), kmin, kmax);
+                store16_part(base + o, window16(rowblk, o, kBlockB), kmin, kmax);
             }
         }
     }
@@ -508,29 +522,35 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // how many CTAs of them fit on an SM.
 constexpr int kMaxDevices = 128;
 std::mutex g_inv_mu;
-int g_inv_grid[kMaxDevices];   // SMs x resident CTAs, 0 until set up
+int g_inv_grid[kMaxDevices][2];   // SMs x resident CTAs (8-warp, narrow instance), 0 until set up
 
-cudaError_t inverse_grid_cap(int *cap) {
+cudaError_t inverse_grid_cap(bool narrow, int *cap) {
     int dev = 0;
     if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_inv_mu);
-    if (g_inv_grid[dev] == 0) {
-        int sms = 0, occ_m = 0, occ_k = 0;
+    if (g_inv_grid[dev][0] == 0) {
+        int sms = 0, occ_m = 0, occ_k = 0, occ_n = 0;
         const cudaError_t steps[] = {
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev),
-            cudaFuncSetAttribute(unrearrange_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kInvSmemBytes),
-            cudaFuncSetAttribute(unrearrange_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kInvSmemBytes),
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_m, unrearrange_kernel<true>, kThreads, kInvSmemBytes),
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_k, unrearrange_kernel<false>, kThreads, kInvSmemBytes),
+            cudaFuncSetAttribute(unrearrange_kernel<true, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kInvSmemBytes),
+            cudaFuncSetAttribute(unrearrange_kernel<false, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kInvSmemBytes),
+            cudaFuncSetAttribute(unrearrange_kernel<true, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kInvNarrowSmemBytes),
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_m, unrearrange_kernel<true, 8>, kThreads, kInvSmemBytes),
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_k, unrearrange_kernel<false, 8>, kThreads, kInvSmemBytes),
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_n, unrearrange_kernel<true, 4>, 128, kInvNarrowSmemBytes),
         };
         for (cudaError_t e : steps)
             if (e != cudaSuccess) return e;
         const int occ = occ_m < occ_k ? occ_m : occ_k;
-        if (occ < 1 || sms < 1) return cudaErrorInvalidConfiguration;
-        g_inv_grid[dev] = sms * occ;
+        if (occ < 1 || occ_n < 1 || sms < 1) return cudaErrorInvalidConfiguration;
+        g_inv_grid[dev][0] = sms * occ;
+        g_inv_grid[dev][1] = sms * occ_n;
     }
-    *cap = g_inv_grid[dev];
+    *cap = g_inv_grid[dev][narrow ? 1 : 0];
     return cudaSuccess;
 }
 
@@ -559,18 +579,21 @@ mx_status unrearrange(mx_group_dim dim, const uint8_t *blocked, int64_t rows, in
     const int64_t bound = dim_m ? (ceil_div(rows, 128) + G) * s.col_chunks
                                 : ceil_div(rows, 128) * (ceil_div(cols, kChunkCols) + G);
     if (bound > INT_MAX) return MX_ERR_UNSUPPORTED;
-    int cap = 0;
-    if (cudaError_t e = inverse_grid_cap(&cap); e != cudaSuccess) return mx_record_cuda_error(e);
-    const int grid = (int)(bound < 1 ? 1 : (bound < cap ? bound : cap));
-    const int64_t blocked_size = (int64_t)mx_rearranged_size(dim, rows, cols, G);
     // flat mode: rows back to back, one item per row block, whole words
     const int mode = dim_m && row_stride == cols && cols <= kTilesPerChunk * 4 && cols % 4 == 0 ? kModeFlat
                      : (row_stride & 15) == 0                                                  ? kModeShift
                                                                                                 : kModeRows;
-    cudaError_t e = dim_m ? launch_pdl(unrearrange_kernel<true>, grid, kThreads, kInvSmemBytes, stream, blocked,
-                                       blocked_size, ends, scales, row_stride, s, mode)
-                          : launch_pdl(unrearrange_kernel<false>, grid, kThreads, kInvSmemBytes, stream, blocked,
-                                       blocked_size, ends, scales, row_stride, s, mode);
+    const bool narrow = mode == kModeFlat && s.padded_cols <= kInvNarrowCols;
+    int cap = 0;
+    if (cudaError_t e = inverse_grid_cap(narrow, &cap); e != cudaSuccess) return mx_record_cuda_error(e);
+    const int grid = (int)(bound < 1 ? 1 : (bound < cap ? bound : cap));
+    const int64_t blocked_size = (int64_t)mx_rearranged_size(dim, rows, cols, G);
+    cudaError_t e = narrow  ? launch_pdl(unrearrange_kernel<true, 4>, grid, 128, kInvNarrowSmemBytes, stream, blocked,
+                                         blocked_size, ends, scales, row_stride, s, mode)
+                    : dim_m ? launch_pdl(unrearrange_kernel<true, 8>, grid, kThreads, kInvSmemBytes, stream, blocked,
+                                         blocked_size, ends, scales, row_stride, s, mode)
+                            : launch_pdl(unrearrange_kernel<false, 8>, grid, kThreads, kInvSmemBytes, stream, blocked,
+                                         blocked_size, ends, scales, row_stride, s, mode);
     return e == cudaSuccess ? MX_OK : mx_record_cuda_error(e);
 }
 
