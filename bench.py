@@ -122,15 +122,16 @@ def load_peaks():
 
 
 FORWARD_SOURCES = ("mx_device.cuh", "mx_rearrange.cu")   # what the rearrange kernels are built from
+INVERSE_SOURCES = ("mx_device.cuh", "mx_inverse.cu")     # what the inverse kernels are built from
 HOST_MARKER = b"// ------------------------------------------------------------------ host side"
 
 
-def kernel_source_sha(root: str = ROOT) -> str:
-    """sha256 prefix of the forward kernels' device code (mx_device.cuh, and
-    mx_rearrange.cu up to its host-side section)."""
+def kernel_source_sha(root: str = ROOT, op: str = "rearrange") -> str:
+    """sha256 prefix of the device code of the op's kernels (mx_device.cuh, and
+    mx_rearrange.cu or mx_inverse.cu up to its host-side section)."""
     h = hashlib.sha256()
     csrc = os.path.join(root, "scale_factor_layout_b200", "csrc")
-    for name in FORWARD_SOURCES:
+    for name in FORWARD_SOURCES if op == "rearrange" else INVERSE_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             data = f.read()
         cut = data.find(HOST_MARKER)
@@ -139,18 +140,19 @@ def kernel_source_sha(root: str = ROOT) -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str):
-    """DRAM bytes per launch recorded by an ncu capture (profiles/ncu_traffic.txt),
-    or None when absent or taken on different kernel sources."""
+def ncu_traffic(call: str, op: str = "rearrange"):
+    """DRAM bytes per launch recorded by an ncu capture (profiles/ncu_traffic.txt)
+    of the op's kernel for this call, or None when absent or taken on different
+    kernel sources."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
-    sha = kernel_source_sha()
+    sha = kernel_source_sha(op=op)
     for line in open(path):
         if line.startswith("#") or not line.strip():
             continue
         kv = dict(tok.split("=", 1) for tok in line.split() if "=" in tok)
-        if kv.get("call") == kernel and kv.get("source_sha") == sha:
+        if kv.get("op", "rearrange") == op and kv.get("call") == call and kv.get("source_sha") == sha:
             return int(float(kv["bytes_per_launch"]))
     return None
 
@@ -431,7 +433,7 @@ def run_ours(args, rank, world, local):
     roofline = {"bound": "hbm", "kernel": f"{kname} ({dc['case']})",
                 "achieved": round(achieved / avg[dom] / 1e9, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / avg[dom] / 1e9 / peak, 4), "peak_source": f"{peak_src} hbm_gbs",
-                "traffic": ncu_traffic(dc["case"]) if args.op == "rearrange" else None,
+                "traffic": ncu_traffic(dc["case"], args.op),
                 "algorithmic_bytes": achieved}
 
     if args.op == "inverse":

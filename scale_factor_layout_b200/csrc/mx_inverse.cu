@@ -499,6 +499,8 @@ __global__ void padded_starts_kernel(const int32_t *__restrict__ ends, int32_t *
     for (int g = threadIdx.x; g <= s.G; g += 32) starts[g] = g < s.G ? table.pstart[g] : table.pstart[kMaxGroups];
 }
 
+// ------------------------------------------------------------------ host side
+
 constexpr int64_t kMaxExtent = (1ll << 31) - (1ll << 14);
 
 template <typename... KArgs, typename... Args>
