@@ -503,18 +503,18 @@ __global__ void padded_starts_kernel(const int32_t *__restrict__ ends, int32_t *
 
 constexpr int64_t kMaxExtent = (1ll << 31) - (1ll << 14);
 
+// A plain stream-ordered launch, as in mx_rearrange.cu (no programmatic
+// stream serialization: it cost time at every switch between kernels).
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, int smem, cudaStream_t stream, Args... args) {
+cudaError_t launch_kernel(void (*kernel)(KArgs...), int grid, int block, int smem, cudaStream_t stream,
+                          Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
@@ -590,11 +590,11 @@ mx_status unrearrange(mx_group_dim dim, const uint8_t *blocked, int64_t rows, in
     if (cudaError_t e = inverse_grid_cap(narrow, &cap); e != cudaSuccess) return mx_record_cuda_error(e);
     const int grid = (int)(bound < 1 ? 1 : (bound < cap ? bound : cap));
     const int64_t blocked_size = (int64_t)mx_rearranged_size(dim, rows, cols, G);
-    cudaError_t e = narrow  ? launch_pdl(unrearrange_kernel<true, 4>, grid, 128, kInvNarrowSmemBytes, stream, blocked,
+    cudaError_t e = narrow  ? launch_kernel(unrearrange_kernel<true, 4>, grid, 128, kInvNarrowSmemBytes, stream, blocked,
                                          blocked_size, ends, scales, row_stride, s, mode)
-                    : dim_m ? launch_pdl(unrearrange_kernel<true, 8>, grid, kThreads, kInvSmemBytes, stream, blocked,
+                    : dim_m ? launch_kernel(unrearrange_kernel<true, 8>, grid, kThreads, kInvSmemBytes, stream, blocked,
                                          blocked_size, ends, scales, row_stride, s, mode)
-                            : launch_pdl(unrearrange_kernel<false, 8>, grid, kThreads, kInvSmemBytes, stream, blocked,
+                            : launch_kernel(unrearrange_kernel<false, 8>, grid, kThreads, kInvSmemBytes, stream, blocked,
                                          blocked_size, ends, scales, row_stride, s, mode);
     return e == cudaSuccess ? MX_OK : mx_record_cuda_error(e);
 }
@@ -637,8 +637,8 @@ mx_status mx_padded_group_starts(mx_group_dim dim, int64_t rows, int64_t cols, c
     if (group_end_offsets == nullptr || starts == nullptr) return MX_ERR_INVALID_ARG;
     const mx::Shape s = mx::make_shape(rows, cols, num_groups);
     cudaError_t e = dim == MX_GROUPS_M
-                        ? mx::launch_pdl(mx::padded_starts_kernel<true>, 1, 32, 0, stream, group_end_offsets, starts, s)
-                        : mx::launch_pdl(mx::padded_starts_kernel<false>, 1, 32, 0, stream, group_end_offsets, starts,
+                        ? mx::launch_kernel(mx::padded_starts_kernel<true>, 1, 32, 0, stream, group_end_offsets, starts, s)
+                        : mx::launch_kernel(mx::padded_starts_kernel<false>, 1, 32, 0, stream, group_end_offsets, starts,
                                          s);
     return e == cudaSuccess ? MX_OK : mx_record_cuda_error(e);
 }
