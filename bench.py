@@ -24,6 +24,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -128,15 +129,18 @@ HOST_MARKER = b"// -------------------------------------------------------------
 
 def kernel_source_sha(root: str = ROOT, op: str = "rearrange") -> str:
     """sha256 prefix of the device code of the op's kernels (mx_device.cuh, and
-    mx_rearrange.cu or mx_inverse.cu up to its host-side section)."""
+    mx_rearrange.cu or mx_inverse.cu up to its host-side section), with `//`
+    comments and blank lines left out so that comment edits keep the key."""
     h = hashlib.sha256()
     csrc = os.path.join(root, "scale_factor_layout_b200", "csrc")
     for name in FORWARD_SOURCES if op == "rearrange" else INVERSE_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             data = f.read()
         cut = data.find(HOST_MARKER)
+        code = data if cut < 0 else data[:cut]
+        lines = (re.sub(rb"//.*", b"", ln).rstrip() for ln in code.split(b"\n"))
         h.update(name.encode())
-        h.update(data if cut < 0 else data[:cut])
+        h.update(b"\n".join(ln for ln in lines if ln))
     return h.hexdigest()[:16]
 
 

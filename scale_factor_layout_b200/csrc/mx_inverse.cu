@@ -3,10 +3,13 @@
 //
 // The blocked layout is the one of mx_rearrange.cu (pytorch/ao #3604: each
 // group made of 128x4 scale-factor tiles; #3285: padded group starts are a
-// prefix sum of padded sizes, computed in the kernel).  The inverse reads a
-// work item's tiles as whole 512-byte lines (one warp reads one tile per
-// 128-bit load), transposes 4x4 words in registers, and writes 16-byte row
-// segments; the padded starts come from the same warp-shuffle scan.
+// prefix sum of padded sizes, computed in the kernel).  The inverse streams a
+// work item's tiles into shared memory with a bulk copy, reads them as whole
+// 512-byte lines (one warp reads one tile per 128-bit load), transposes 4x4
+// words in registers into a shared row block, and writes the output in
+// 16-byte aligned chunks that each have exactly one owning item (partial ones
+// as byte-masked bulk copies); the padded starts come from the same
+// warp-shuffle scan.
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -39,10 +42,11 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes
                  : "memory");
 }
 
-// Shared-memory row block of one work item: 128 rows of up to 36 tiles' columns
-// (the item's 32 tiles and the quad before them) at pitch 144 bytes (9 x 16,
-// odd: conflict-free 16-byte accesses down a column).  In flat mode the rows
-// sit back to back instead (row r at r * cols).
+// Shared-memory row block of one work item: 128 rows of 144 bytes (9 x 16,
+// odd: conflict-free 16-byte accesses down a column), which hold up to 36
+// tiles' columns (the item's 32 tiles and the quad before them) or, in shift
+// mode, the 9 output chunks a row of the item can touch.  In flat mode the
+// rows sit back to back instead (row r at r * cols).
 constexpr int kInvPreTiles = 4;                                         // quad loaded before an item
 constexpr int kInvPitch = (kTilesPerChunk + kInvPreTiles) * 4;          // 144
 constexpr int kInvStages = 2;                                           // items in flight per CTA

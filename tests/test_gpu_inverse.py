@@ -68,6 +68,23 @@ def test_inverse_every_chunk_offset(mxlib, orc, misalign):
     _inverse_check(m_case, orc, out_pad=(-150) % 16, misalign=misalign)
 
 
+@pytest.mark.parametrize("misalign", [0, 1, 5, 11, 13, 15])
+def test_inverse_narrow_k_groups(mxlib, orc, misalign):
+    """K groups of 0..24 columns, so that seam chunks hold bytes of up to three
+    groups and every branch of the seam rule runs: seams written whole by the
+    later group, seams left to masked copies because the earlier group is
+    narrower than the seam offset, because its columns spread over five tiles,
+    or because the later group does not fill the chunk; empty groups between."""
+    rng = np.random.default_rng(4200 + misalign)
+    rows, G = 260, 64
+    widths = rng.integers(0, 25, size=G)
+    widths[rng.random(G) < 0.2] = 0
+    cols = int(widths.sum()) + 7          # the last 7 columns are not covered by any group
+    scales = rng.integers(1, 255, size=(rows, cols), dtype=np.uint8)
+    case = synth.Case("narrowK", synth.DIM_K, scales, np.cumsum(widths).astype(np.int32), 0)
+    _inverse_check(case, orc, out_pad=(-cols) % 16 + 16, misalign=misalign)
+
+
 def test_inverse_sweep_subset(mxlib, orc):
     for i_rows in range(len(synth.SWEEP_ROWS)):
         for i_k in (0, 3, 6):
