@@ -53,12 +53,13 @@ constexpr int kInvStages = 2;                                           // items
 constexpr int kInvStageBytes = (kTilesPerChunk + kInvPreTiles) * 512;   // 18 KB
 constexpr int kInvBlockBytes = kTileRows * kInvPitch;                   // 18 KB
 constexpr int kInvSmemBytes = kInvStages * kInvStageBytes + 2 * kInvBlockBytes + 128;
-// The narrow instance (4 warps) runs flat mode for rows of at most 64 padded
-// columns: an item is at most 16 tiles, its rows at most 8 KB together, so a
-// CTA is small enough that about one row block per CTA is resident at once.
-constexpr int kInvNarrowCols = 64;
-constexpr int kInvNarrowStageBytes = (kInvNarrowCols / 4) * 512;             // 8 KB
-constexpr int kInvNarrowBlockBytes = kTileRows * kInvNarrowCols;             // 8 KB
+// The narrow instance (4 warps) runs flat mode for rows of at most 48 padded
+// columns: an item is at most 12 tiles, its rows at most 6 KB together, so 7
+// CTAs fit on an SM and about one row block per CTA is resident at once
+// (1032 row blocks of a 131072-row input, 1036 CTAs on a B200).
+constexpr int kInvNarrowCols = 48;
+constexpr int kInvNarrowStageBytes = (kInvNarrowCols / 4) * 512;             // 6 KB
+constexpr int kInvNarrowBlockBytes = kTileRows * kInvNarrowCols;             // 6 KB
 constexpr int kInvNarrowSmemBytes = kInvStages * kInvNarrowStageBytes + 2 * kInvNarrowBlockBytes + 128;
 constexpr uint32_t kInvFlagWaitTimeout = 1u;
 
@@ -251,7 +252,7 @@ constexpr int kModeFlat = 2;    // rows back to back (stride == cols <= 128)
 //     (rows back to back in memory): the item's rows are one contiguous span
 //     and threads take its chunks in order.
 template <bool kDimM, int kWarpsI>
-__global__ void __launch_bounds__(kWarpsI * 32, kWarpsI == 8 ? 3 : 6)
+__global__ void __launch_bounds__(kWarpsI * 32, kWarpsI == 8 ? 3 : 7)
 unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, const int32_t *__restrict__ ends,
                    uint8_t *__restrict__ scales, int64_t row_stride, Shape s, int mode) {
     static_assert(kWarpsI == 8 || kWarpsI == 4, "8 warps (every mode) or 4 (narrow flat rows)");
@@ -259,7 +260,7 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
     constexpr int kThr = kWarpsI * 32;
     constexpr int kStageB = kNarrow ? kInvNarrowStageBytes : kInvStageBytes;
     constexpr int kBlockB = kNarrow ? kInvNarrowBlockBytes : kInvBlockBytes;
-    constexpr int kPasses = kNarrow ? 1 : 2;   // quads of tiles per thread (at most 4, or 9)
+    constexpr int kPasses = kNarrow ? 1 : 2;   // quads of tiles per thread (at most 3, or 9)
     extern __shared__ uint8_t dyn_smem[];
     uint8_t *stages = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 127) & ~uintptr_t(127));
     uint8_t *rowblks = stages + kInvStages * kStageB;
