@@ -104,21 +104,26 @@ rearrange_tma_m(const __grid_constant__ CUtensorMap tmap, const int32_t *__restr
     const int bid = blockIdx.x;
     const int n_my = bid < total ? (total - 1 - bid) / (int)gridDim.x + 1 : 0;
 
-    auto issue = [&](int n, int st) {
-        const Item it = decode_item<true>(table, s, bid + n * (int)gridDim.x, 16);
+    auto decode = [&](int n) { return decode_item<true>(table, s, bid + n * (int)gridDim.x, 16); };
+    auto issue = [&](const Item &it, int st) {
         items[st] = it;
         mbar_arrive_expect_tx(&full[st], kStageBytes);
         tma_load_2d(stages + st * kStageBytes, &tmap, it.x, it.y, &full[st]);
     };
 
     if (tid == 0)
-        for (int st = 0; st < kStages && st < n_my; ++st) issue(st, st);
+        for (int st = 0; st < kStages && st < n_my; ++st) issue(decode(st), st);
 
     int64_t prev_off = 0;     // thread 0: output span of the previous item
     uint32_t prev_bytes = 0;
     for (int n = 0; n < n_my; ++n) {
         const int st = n % kStages;
         const uint32_t parity = (uint32_t)(n / kStages) & 1u;
+        // Thread 0 decodes the stage's refill while its current load is in
+        // flight; after the barrier it issues that load before anything else.
+        const bool refill = tid == 0 && n + kStages < n_my;
+        Item next;
+        if (refill) next = decode(n + kStages);
         const bool ok = mbar_wait_bounded(&full[st], parity);
         uint4 w[4];
         Item it;
@@ -140,13 +145,13 @@ rearrange_tma_m(const __grid_constant__ CUtensorMap tmap, const int32_t *__restr
             return;
         }
         if (tid == 0) {
+            if (refill) issue(next, st);
             if (n > 0) {
                 bulk_store_s2g(out + prev_off, staging + ((n - 1) & 1) * kOutBytes, prev_bytes);
                 bulk_commit();
             }
             prev_off = it.out_off;
             prev_bytes = (uint32_t)it.ntiles * 512u;
-            if (n + kStages < n_my) issue(n + kStages, st);
         }
         mask_and_stage(w, it, j, q, staging + (n & 1) * kOutBytes);
         fence_proxy_async_smem();
@@ -227,7 +232,7 @@ rearrange_tma_k(const __grid_constant__ CUtensorMap tmap, const int32_t *__restr
     const int bid = blockIdx.x;
     const int n_my = bid < total ? (total - 1 - bid) / (int)gridDim.x + 1 : 0;
 
-    auto issue = [&](int n, int st) {
+    auto decode = [&](int n) {
         const int i = bid + n * (int)gridDim.x;
         KItem it;
         it.rb = i / per_band;
@@ -239,6 +244,9 @@ rearrange_tma_k(const __grid_constant__ CUtensorMap tmap, const int32_t *__restr
         it.y = it.rb * kTileRows;
         it.rows_valid = min(kTileRows, s.rows - it.y);
         it.pad = 0;
+        return it;
+    };
+    auto issue = [&](const KItem &it, int st) {
         items[st] = it;
         mbar_arrive_expect_tx(&full[st], kStageBytes);
         tma_load_2d(stages + st * kStageBytes, &tmap, it.x, it.y, &full[st]);
@@ -262,13 +270,17 @@ rearrange_tma_k(const __grid_constant__ CUtensorMap tmap, const int32_t *__restr
     };
 
     if (tid == 0)
-        for (int st = 0; st < kStages && st < n_my; ++st) issue(st, st);
+        for (int st = 0; st < kStages && st < n_my; ++st) issue(decode(st), st);
 
     KItem prev;
     prev.ntiles = 0;
     for (int n = 0; n < n_my; ++n) {
         const int st = n % kStages;
         const uint32_t parity = (uint32_t)(n / kStages) & 1u;
+        // the stage's refill is decoded while its current load is in flight
+        const bool refill = tid == 0 && n + kStages < n_my;
+        KItem next;
+        if (refill) next = decode(n + kStages);
         const bool ok = mbar_wait_bounded(&full[st], parity);
         uint4 w[4] = {};
         uint32_t cm[4] = {0u, 0u, 0u, 0u};
@@ -325,9 +337,9 @@ rearrange_tma_k(const __grid_constant__ CUtensorMap tmap, const int32_t *__restr
             return;
         }
         if (tid == 0) {
+            if (refill) issue(next, st);
             if (n > 0) store_item(prev, staging + ((n - 1) & 1) * kOutBytes);
             prev = it;
-            if (n + kStages < n_my) issue(n + kStages, st);
         }
         // masked lines of this thread's tiles into staging block n % 2
         {
@@ -431,7 +443,7 @@ rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__re
     const int bid = blockIdx.x;
     const int n_my = bid < total ? (total - 1 - bid) / (int)gridDim.x + 1 : 0;
 
-    auto issue = [&](int n, int st) {
+    auto decode = [&](int n) {
         const int i = bid + n * (int)gridDim.x;
         const int g = find_group(table, s.G, i);
         const int rb = i - table.istart[g];
@@ -444,8 +456,11 @@ rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__re
         const int64_t byte0 = (int64_t)it.y * L;
         const int64_t word0 = (byte0 >> 4) << 2;
         it.delta = (int)(byte0 - word0 * 4);
-        const int nbox = (it.delta + it.rows_valid * L + kFlatBoxBytes - 1) / kFlatBoxBytes;
         it.x = (int)word0;
+        return it;
+    };
+    auto issue = [&](const Item &it, int st) {
+        const int nbox = (it.delta + it.rows_valid * L + kFlatBoxBytes - 1) / kFlatBoxBytes;
         items[st] = it;
         mbar_arrive_expect_tx(&full[st], (uint32_t)nbox * kFlatBoxBytes);
         for (int b = 0; b < nbox; ++b)
@@ -453,13 +468,17 @@ rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__re
     };
 
     if (tid == 0)
-        for (int st = 0; st < kStagesF && st < n_my; ++st) issue(st, st);
+        for (int st = 0; st < kStagesF && st < n_my; ++st) issue(decode(st), st);
 
     int64_t prev_off = 0;
     uint32_t prev_bytes = 0;
     for (int n = 0; n < n_my; ++n) {
         const int st = n % kStagesF;
         const uint32_t parity = (uint32_t)(n / kStagesF) & 1u;
+        // the stage's refill is decoded while its current load is in flight
+        const bool refill = tid == 0 && n + kStagesF < n_my;
+        Item next;
+        if (refill) next = decode(n + kStagesF);
         const bool ok = mbar_wait_bounded(&full[st], parity);
         Item it;
         uint32_t wv[kPasses][4][4];   // [quad pass][row a][word t]
@@ -487,13 +506,13 @@ rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__re
             return;
         }
         if (tid == 0) {
+            if (refill) issue(next, st);
             if (n > 0) {
                 bulk_store_s2g(out + prev_off, staging + ((n - 1) & 1) * f.staging_bytes, prev_bytes);
                 bulk_commit();
             }
             prev_off = it.out_off;
             prev_bytes = (uint32_t)it.ntiles * 512u;
-            if (n + kStagesF < n_my) issue(n + kStagesF, st);
         }
         uint8_t *stg = staging + (n & 1) * f.staging_bytes;
 #pragma unroll
