@@ -11,7 +11,8 @@
 //     #3708, "fallback cuda kernel for when input doesn't meet 2d TMA
 //     constraints", Context).
 //   * rearrange_flat_tma: M-groups with narrow rows whose stride is a multiple
-//     of 4: 1-D TMA boxes over whole row blocks.
+//     of 4: 1-D TMA boxes over whole row blocks (an 8-warp instance, and a
+//     4-warp one for rows of at most 64 padded columns).
 //   * rearrange_fallback: work items loaded with ordinary 32-bit (or byte)
 //     loads, for any stride or alignment (#3708's fallback).
 // Every CTA scans the group ends itself (#3285, "compute prefix sum of group
@@ -53,8 +54,9 @@ constexpr int tma_smem_bytes() { return kStages * stage_bytes<kDimM>() + kOutBuf
 //      per thread into registers;
 //   2. one barrier: the stage and the staging block n % 2 are free, and the
 //      staging block of item n-1 is complete;
-//   3. thread 0 bulk-stores item n-1's tiles (shared -> global, asynchronous)
-//      and refills the stage with the TMA load of item n + kStages;
+//   3. thread 0 refills the stage with the TMA load of item n + kStages
+//      (decoded while the stage's load was in flight) and then bulk-stores
+//      item n-1's tiles (shared -> global, asynchronous);
 //   4. every thread writes its masked output lines of item n into staging.
 // Loads and stores are both asynchronous copies driven by one thread, so the
 // 8 warps only move data between shared memory and registers.
