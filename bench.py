@@ -297,7 +297,7 @@ def rotation_count(case) -> int:
     return max(2, math.ceil(4 * L2_BYTES / (b["read"] + b["alloc"])))
 
 
-def launch(item, stream_handle, op="rearrange"):
+def launch(item, stream_handle, op="rearrange", path="auto"):
     from scale_factor_layout_b200 import _binding as B
 
     c, s, e, o = item
@@ -306,7 +306,7 @@ def launch(item, stream_handle, op="rearrange"):
         st = fn(s.data_ptr(), c.rows, c.cols, e.data_ptr(), c.num_groups, o.data_ptr(), c.cols, stream_handle)
     else:
         st = B.mx_rearrange_ex(c.dim, s.data_ptr(), c.rows, c.cols, c.cols, e.data_ptr(), c.num_groups,
-                               o.data_ptr(), B.MX_PATH_AUTO, stream_handle)
+                               o.data_ptr(), B.PATHS[path], stream_handle)
     if st != B.MX_OK:
         raise RuntimeError(f"{c.name}: {B.status_string(st)}")
 
@@ -340,7 +340,7 @@ def run_ours(args, rank, world, local):
     with torch.cuda.stream(stream):
         for k in range(3):  # first calls set kernel attributes (outside capture) and warm caches
             for it in step_items(k):
-                launch(it, h, args.op)
+                launch(it, h, args.op, args.path)
     torch.cuda.synchronize()
 
     def capture(launches):
@@ -349,7 +349,7 @@ def run_ours(args, rank, world, local):
         with torch.cuda.stream(stream):
             with torch.cuda.graph(g, stream=stream):
                 for it in launches:
-                    launch(it, h, args.op)
+                    launch(it, h, args.op, args.path)
         return g
 
     def steps_of(k0, n):
@@ -418,7 +418,8 @@ def run_ours(args, rank, world, local):
     calls = []
     for ci, (c, b, t) in enumerate(zip(cases, per_call, avg)):
         gbs = (b["read"] + b["written"]) / t / 1e9
-        path = mxs.mx_select_path(c.dim, rot[cases.index(c)][0][1].data_ptr(), c.rows, c.cols, c.cols)
+        path = (mxs.mx_select_path(c.dim, rot[cases.index(c)][0][1].data_ptr(), c.rows, c.cols, c.cols)
+                if args.path == "auto" else B.PATHS[args.path])
         calls.append({"case": c.name, "path": B.PATH_NAMES.get(path, "?"),
                       "us": round(t * 1e6, 3), "gbps": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
                       "read_bytes": b["read"], "written_bytes": b["written"], "alloc_bytes": b["alloc"],
@@ -437,19 +438,21 @@ def run_ours(args, rank, world, local):
     roofline = {"bound": "hbm", "kernel": f"{kname} ({dc['case']})",
                 "achieved": round(achieved / avg[dom] / 1e9, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / avg[dom] / 1e9 / peak, 4), "peak_source": f"{peak_src} hbm_gbs",
-                "traffic": ncu_traffic(dc["case"], args.op),
+                "traffic": ncu_traffic(dc["case"], args.op) if args.path == "auto" else None,
                 "algorithmic_bytes": achieved}
 
     if args.op == "inverse":
         for cl in calls:
             cl["path"] = "inverse"
-    e2e = run_e2e(args, cases, device, world, dist) if not args.no_e2e and args.op == "rearrange" else None
+    e2e = (run_e2e(args, cases, device, world, dist)
+           if not args.no_e2e and args.op == "rearrange" and args.path == "auto" else None)
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(seconds_max / args.steps * 1e3, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
         "data": "synthetic (seeded uniform E8M0 bytes, seeded group splits)",
-        "config": {"workload": args.workload, "op": args.op, "description": workload_desc(args.workload),
+        "config": {"workload": args.workload, "op": args.op, "path": args.path,
+                   "description": workload_desc(args.workload),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "bytes_per_step": step_bytes, "bytes_per_step_pages_convention": step_bytes_pages,
                    "l2": "inputs/outputs rotate per call over " + ", ".join(str(len(r)) for r in rot)
@@ -632,7 +635,8 @@ def run_reference(args, rank, world):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(seconds / args.steps * 1e3, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
            "data": "synthetic (seeded uniform E8M0 bytes, seeded group splits)",
-           "config": {"workload": args.workload, "op": args.op, "description": workload_desc(args.workload),
+           "config": {"workload": args.workload, "op": args.op, "path": args.path,
+                      "description": workload_desc(args.workload),
                       "parallelism": "single host thread"},
            "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
                             "sample": f"{desc}, single thread, gcc -O2, {cpu_model()}"},
@@ -650,6 +654,8 @@ def main(argv=None):
                     help=f"one of {sorted(WORKLOADS)} or k_sweep_<M>x<TotalK> (a point of the K-groups sweep)")
     ap.add_argument("--op", choices=["rearrange", "inverse"], default="rearrange",
                     help="rearrange (row-major -> blocked, the hot path) or its inverse")
+    ap.add_argument("--path", choices=["auto", "tma", "flat", "word", "byte"], default="auto",
+                    help="force one kernel path of the rearrange, to measure the others (no e2e, no traffic)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
