@@ -657,7 +657,7 @@ def main(argv=None):
     ap.add_argument("--path", choices=["auto", "tma", "flat", "word", "byte"], default="auto",
                     help="force one kernel path of the rearrange, to measure the others (no e2e, no traffic)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=60)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-copy-ceiling", action="store_true",
                     help="skip timing a same-size device-to-device copy per call")
