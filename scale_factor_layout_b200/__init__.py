@@ -10,7 +10,7 @@ torch's current CUDA stream.
 from __future__ import annotations
 
 from ._binding import (  # noqa: F401
-    MX_GROUPS_K, MX_GROUPS_M, MX_MAX_GROUPS, MX_OK, MX_PATH_AUTO, MX_PATH_BYTE, MX_PATH_TMA,
+    MX_GROUPS_K, MX_GROUPS_M, MX_MAX_GROUPS, MX_OK, MX_PATH_AUTO, MX_PATH_BYTE, MX_PATH_FLAT, MX_PATH_TMA,
     MX_PATH_WORD, PATHS, MxError, declared_symbols, lib, mx_device_flags, mx_rearrange_ex,
     mx_rearrange_k_groups, mx_rearrange_m_groups, mx_rearranged_size, mx_select_path,
     mx_padded_group_starts, mx_selftest_bounded_wait, mx_unrearrange_k_groups, mx_unrearrange_m_groups,
@@ -82,13 +82,16 @@ def unrearrange(dim: int, blocked, rows: int, cols: int, group_end_offsets, out=
 
     if blocked.dtype != torch.uint8 or not blocked.is_contiguous() or not blocked.is_cuda:
         raise ValueError("blocked must be a contiguous CUDA uint8 tensor")
-    if group_end_offsets.dtype != torch.int32 or not group_end_offsets.is_cuda:
-        raise ValueError("group_end_offsets must be a CUDA int32 tensor")
+    if group_end_offsets.dtype != torch.int32 or not group_end_offsets.is_cuda or not group_end_offsets.is_contiguous():
+        raise ValueError("group_end_offsets must be a contiguous CUDA int32 tensor")
     G = group_end_offsets.numel()
     if blocked.numel() < mx_rearranged_size(dim, rows, cols, G):
         raise ValueError("blocked is smaller than the layout's allocation")
     if out is None:
         out = torch.empty((rows, cols), dtype=torch.uint8, device=blocked.device)
+    elif (out.dtype != torch.uint8 or out.dim() != 2 or tuple(out.shape) != (rows, cols) or not out.is_cuda
+          or (rows > 1 and cols > 1 and out.stride(1) != 1)):
+        raise ValueError(f"out must be a CUDA uint8 tensor of shape ({rows}, {cols}), dense along columns")
     stride = out.stride(0) if rows > 1 else cols
     if stream is None:
         stream = torch.cuda.current_stream(blocked.device).cuda_stream
@@ -103,6 +106,10 @@ def padded_group_starts(dim: int, rows: int, cols: int, group_end_offsets, strea
     """int32[G + 1] padded group starts (rows for M, columns for K), computed on the GPU."""
     import torch
 
+    if group_end_offsets.dtype != torch.int32 or group_end_offsets.dim() != 1 or not group_end_offsets.is_cuda:
+        raise ValueError("group_end_offsets must be a 1-D CUDA int32 tensor")
+    if not group_end_offsets.is_contiguous():
+        raise ValueError("group_end_offsets must be contiguous")
     G = group_end_offsets.numel()
     starts = torch.empty(G + 1, dtype=torch.int32, device=group_end_offsets.device)
     if stream is None:

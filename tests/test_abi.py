@@ -102,3 +102,20 @@ def test_padded_starts_host_validation(mxlib):
     assert B.mx_padded_group_starts(B.MX_GROUPS_M, 10, 10, 0, 2, 0x1000, 0) == B.MX_ERR_INVALID_ARG
     assert B.mx_padded_group_starts(B.MX_GROUPS_M, 10, 10, 0x1000, 0, 0x2000, 0) == B.MX_ERR_INVALID_ARG
     assert B.mx_padded_group_starts(7, 10, 10, 0x1000, 2, 0x2000, 0) == B.MX_ERR_INVALID_ARG
+
+
+def test_torch_wrappers_reject_bad_tensors():
+    """The torch-level wrappers check their tensors before any library call."""
+    import torch
+
+    import scale_factor_layout_b200 as mxs
+
+    ends = torch.tensor([10, 20], dtype=torch.int32)
+    with pytest.raises(ValueError):   # not on a CUDA device
+        mxs.rearrange(mxs.MX_GROUPS_M, torch.zeros((20, 8), dtype=torch.uint8), ends)
+    with pytest.raises(ValueError):   # wrong dtype
+        mxs.rearrange(mxs.MX_GROUPS_M, torch.zeros((20, 8), dtype=torch.int32), ends)
+    with pytest.raises(ValueError):   # blocked buffer not on a CUDA device
+        mxs.unrearrange(mxs.MX_GROUPS_M, torch.zeros(4096, dtype=torch.uint8), 20, 8, ends)
+    with pytest.raises(ValueError):   # offsets of the wrong dtype
+        mxs.padded_group_starts(mxs.MX_GROUPS_M, 20, 8, torch.tensor([10, 20], dtype=torch.int64))
