@@ -122,9 +122,10 @@ mx_status mx_rearrange_ex(mx_group_dim dim, const uint8_t *scales, int64_t rows,
  * ends) and write the row-major scales: element (i, j) at
  * scales[i * row_stride + j], any alignment.  Elements that no group covers
  * (rows at or past the last clamped end) are written as 0; bytes between
- * cols and row_stride are not touched.  Padding bytes of `blocked` are not
- * read.  Same limits, clamping and stream rules as the forward call; the
- * blocked buffer must not overlap `scales`.  (The other side of the layout
+ * cols and row_stride are not touched.  The values of `blocked`'s padding
+ * bytes do not matter (whole tiles are read, padding included, and ignored).
+ * Same limits, clamping and stream rules as the forward call; the blocked
+ * buffer must not overlap `scales`.  (The other side of the layout
  * the pytorch/ao pages convert to: #3604, 128x4 tiles in each group.) */
 mx_status mx_unrearrange_m_groups(const uint8_t *blocked, int64_t rows, int64_t cols,
                                   const int32_t *group_end_offsets, int32_t num_groups, uint8_t *scales,

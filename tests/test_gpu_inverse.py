@@ -85,6 +85,25 @@ def test_inverse_narrow_k_groups(mxlib, orc, misalign):
     _inverse_check(case, orc, out_pad=(-cols) % 16 + 16, misalign=misalign)
 
 
+def test_inverse_ignores_padding_values(mxlib, orc):
+    """Padding bytes of the blocked buffer (and its tail) filled with garbage
+    change nothing: the inverse reads whole tiles but writes only real data."""
+    rng = np.random.default_rng(4400)
+    cases = [synth.m_tiny(), synth.k_sweep_point(2, 3), synth.random_small(601), synth.random_small(777)]
+    rows, cols = 300, 700
+    cuts = np.sort(rng.choice(np.arange(1, cols), size=7, replace=False))
+    cases.append(synth.Case("padK", synth.DIM_K, rng.integers(1, 255, size=(rows, cols), dtype=np.uint8),
+                            np.append(cuts, cols).astype(np.int32), 0))
+    for case in cases:
+        blocked = orc.rearrange(case.dim, case.scales, case.ends)
+        r, _ = orc.decode_at(case.dim, case.rows, case.cols, case.ends, np.arange(blocked.size, dtype=np.int64))
+        dirty = blocked.copy()
+        pad = r < 0
+        dirty[pad] = rng.integers(1, 256, size=int(pad.sum()), dtype=np.uint8)
+        for pad_out, misalign in ((0, 0), ((-case.cols) % 16 + 16, 3)):
+            _inverse_check(case, orc, out_pad=pad_out, misalign=misalign, blocked_np=dirty)
+
+
 def test_inverse_sweep_subset(mxlib, orc):
     for i_rows in range(len(synth.SWEEP_ROWS)):
         for i_k in (0, 3, 6):
