@@ -15,13 +15,17 @@
 #include <cuda_runtime.h>
 
 #include <climits>
+#include <cstring>
 #include <mutex>
 
 #include "mx_device.cuh"
 #include "mxscale.h"
 
-// Defined in mx_rearrange.cu: note a CUDA failure for mx_last_cuda_error().
+// Defined in mx_rearrange.cu: note a CUDA failure for mx_last_cuda_error(),
+// and encode a 2-D uint8 tensor map over row-major rows.
 mx_status mx_record_cuda_error(cudaError_t e);
+mx_status mx_encode_rows_map(CUtensorMap *map, const void *base, int64_t width, int64_t rows, int64_t row_stride,
+                             uint32_t box_w, uint32_t box_h, CUtensorMapSwizzle swizzle);
 
 namespace mx {
 namespace {
@@ -42,6 +46,15 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes
                  : "memory");
 }
 
+// 2-D tensor store of one box from shared memory (128B-swizzled, 1024-byte
+// aligned) at tensor coordinates (x, y); elements outside the tensor are not
+// written.  Tracked in the issuing thread's bulk groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+
 // Shared-memory row block of one work item: 128 rows of 144 bytes (9 x 16,
 // odd: conflict-free 16-byte accesses down a column), which hold up to 36
 // tiles' columns (the item's 32 tiles and the quad before them) or, in shift
@@ -53,6 +66,7 @@ constexpr int kInvStages = 2;                                           // items
 constexpr int kInvStageBytes = (kTilesPerChunk + kInvPreTiles) * 512;   // 18 KB
 constexpr int kInvBlockBytes = kTileRows * kInvPitch;                   // 18 KB
 constexpr int kInvSmemBytes = kInvStages * kInvStageBytes + 2 * kInvBlockBytes + 128;
+constexpr int kInvTmaSmemBytes = kInvStages * kInvStageBytes + 2 * kInvBlockBytes + 1024;   // 1024-aligned start
 // The narrow instance (4 warps) runs flat mode for rows of at most 48 padded
 // columns: an item is at most 12 tiles, its rows at most 6 KB together, so 7
 // CTAs fit on an SM and about one row block per CTA is resident at once
@@ -90,7 +104,8 @@ struct InvItem {
     int32_t merge;        // 1 if the item writes the seam chunk before its group whole
     int32_t n2;           // merged seam: tiles of the previous group loaded (<= 4)
     int32_t b0;           // merged seam: byte of the first needed column in the first of them
-    int32_t pad;
+    int32_t tx;           // >= 0 if the item's owned bytes are exactly one tensor-store box (clipped):
+                          // the box's first column in the output tensor map (a multiple of 16)
 };
 
 // Groups along K, shift mode: a 16-byte output chunk that holds the seam
@@ -105,9 +120,11 @@ __device__ __forceinline__ bool seam_whole(int w_prev, int w_next, int ls) {
 
 // `out`, `row_stride`: the row-major output, to tell whether an item's first
 // column can start mid-chunk (only then is the quad before it needed).
-template <bool kDimM>
+// `map_w`: width of the output tensor map (0 without one), whose column 0 is
+// the 16-byte boundary at or below the output's first byte.
+template <bool kDimM, bool kTma>
 __device__ __forceinline__ InvItem decode_inv(const GroupTable &t, const Shape &s, int i, const uint8_t *out,
-                                              int64_t row_stride) {
+                                              int64_t row_stride, int64_t map_w) {
     const Item it = decode_item<kDimM>(t, s, i, 1);
     int k, run, g, rb = 0;   // item's chunk index in its run, the run's column count, group, row band
     if (kDimM) {
@@ -146,7 +163,6 @@ __device__ __forceinline__ InvItem decode_inv(const GroupTable &t, const Shape &
     v.n2 = 0;
     v.b0 = 0;
     v.src2_off = 0;
-    v.pad = 0;
     if (!kDimM && shift) {
         if (k == 0 && v.lead != 0) {
             int gp = g - 1;
@@ -171,6 +187,20 @@ __device__ __forceinline__ InvItem decode_inv(const GroupTable &t, const Shape &
     v.hi = hi_c + v.lead;
     v.nch = (v.hi + 15) >> 4;
     v.partial = ((v.lo & 15) != 0 || (v.hi & 15) != 0) ? 1 : 0;
+    // One tensor store writes a 128 x 128 box, clipped at the map's last row
+    // and at its right edge (in whole 16-byte units): usable when that is
+    // exactly what the item owns.  Groups along M only: for K-groups rows
+    // (4 KB apart at the measured sizes) the tensor store was slower than the
+    // threads' own stores (15.7 vs 15.0 us at 7168x4096; M-groups 131072x224:
+    // 11.4 vs 12.7 us).
+    v.tx = -1;
+    if (kTma && kDimM && shift && map_w > 0 && v.lo == 0) {
+        const int64_t x = (int64_t)it.x + (int64_t)(reinterpret_cast<uintptr_t>(out) & 15u) - v.lead;
+        const bool cols_ok = v.hi == kTilesPerChunk * 4 ? x + kTilesPerChunk * 4 <= map_w
+                                                        : x + v.hi == map_w && (map_w & 15) == 0;
+        const bool rows_ok = v.rows_valid == kTileRows || v.y + v.rows_valid == s.rows;
+        if (cols_ok && rows_ok) v.tx = (int)x;
+    }
     return v;
 }
 
@@ -251,10 +281,11 @@ constexpr int kModeFlat = 2;    // rows back to back (stride == cols <= 128)
 //     window around it, partial ones stored by words and bytes.  Flat mode
 //     (rows back to back in memory): the item's rows are one contiguous span
 //     and threads take its chunks in order.
-template <bool kDimM, int kWarpsI>
-__global__ void __launch_bounds__(kWarpsI * 32, kWarpsI == 8 ? 3 : 7)
-unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, const int32_t *__restrict__ ends,
-                   uint8_t *__restrict__ scales, int64_t row_stride, Shape s, int mode) {
+template <bool kDimM, int kWarpsI, bool kTma>
+__device__ __forceinline__ void unrearrange_body(const CUtensorMap *omap, int64_t map_w,
+                                                 const uint8_t *__restrict__ blocked, int64_t blocked_size,
+                                                 const int32_t *__restrict__ ends, uint8_t *__restrict__ scales,
+                                                 int64_t row_stride, const Shape &s, int mode) {
     static_assert(kWarpsI == 8 || kWarpsI == 4, "8 warps (every mode) or 4 (narrow flat rows)");
     constexpr bool kNarrow = kWarpsI == 4;
     constexpr int kThr = kWarpsI * 32;
@@ -262,7 +293,10 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
     constexpr int kBlockB = kNarrow ? kInvNarrowBlockBytes : kInvBlockBytes;
     constexpr int kPasses = kNarrow ? 1 : 2;   // quads of tiles per thread (at most 3, or 9)
     extern __shared__ uint8_t dyn_smem[];
-    uint8_t *stages = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 127) & ~uintptr_t(127));
+    // 1024-byte aligned where a row block may be the source of a 128B-swizzled
+    // tensor store (stage and row block sizes are multiples of 1 KB)
+    constexpr uintptr_t kAlign = kTma ? 1024 : 128;
+    uint8_t *stages = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + kAlign - 1) & ~(kAlign - 1));
     uint8_t *rowblks = stages + kInvStages * kStageB;
     __shared__ GroupTable table;
     __shared__ __align__(8) uint64_t full[kInvStages];
@@ -295,7 +329,9 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
     const int bid = blockIdx.x;
     const int n_my = bid < total ? (total - 1 - bid) / (int)gridDim.x + 1 : 0;
 
-    auto decode = [&](int n) { return decode_inv<kDimM>(table, s, bid + n * (int)gridDim.x, scales, row_stride); };
+    auto decode = [&](int n) {
+        return decode_inv<kDimM, kTma>(table, s, bid + n * (int)gridDim.x, scales, row_stride, map_w);
+    };
     auto issue = [&](const InvItem &it, int st) {
         items[st] = it;
         const uint32_t bytes = (uint32_t)it.nload * 512u, bytes2 = (uint32_t)it.n2 * 512u;
@@ -343,7 +379,11 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
                     for (int a = 0; a < 4; ++a) {
                         const uint32_t x0 = word_of(w[0], a), x1 = word_of(w[1], a), x2 = word_of(w[2], a),
                                        x3 = word_of(w[3], a), x4 = word_of(w[4], a);
-                        *reinterpret_cast<uint4 *>(rowblk + (j + 32 * a) * kInvPitch + 16 * m) =
+                        // chunk m of row j + 32a: plain rows at pitch kInvPitch, or the
+                        // 128B-swizzled rows of 128 bytes a tensor store reads
+                        *reinterpret_cast<uint4 *>((kTma && it.tx >= 0)
+                                                       ? rowblk + (j + 32 * a) * 128 + 16 * (m ^ (j & 7))
+                                                       : rowblk + (j + 32 * a) * kInvPitch + 16 * m) =
                             make_uint4(funnel(x0, x1, sh), funnel(x1, x2, sh), funnel(x2, x3, sh), funnel(x3, x4, sh));
                     }
                     if (!kDimM && m == 0 && it.merge) {
@@ -365,7 +405,9 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
                         for (int a = 0; a < 4; ++a) {
                             const uint32_t p0 = word_of(w[0], a), p1 = word_of(w[1], a), p2 = word_of(w[2], a),
                                            p3 = word_of(w[3], a);
-                            uint4 *dst = reinterpret_cast<uint4 *>(rowblk + (j + 32 * a) * kInvPitch);
+                            uint4 *dst = reinterpret_cast<uint4 *>((kTma && it.tx >= 0)
+                                                                       ? rowblk + (j + 32 * a) * 128 + 16 * (j & 7)
+                                                                       : rowblk + (j + 32 * a) * kInvPitch);
                             const uint4 own = *dst;
                             *dst = make_uint4((funnel(p0, p1, sh0) & keep[0]) | (own.x & ~keep[0]),
                                               (funnel(p1, p2, sh0) & keep[1]) | (own.y & ~keep[1]),
@@ -374,8 +416,8 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
                         }
                     }
                 }
-                // the masked bulk copies of the store phase read this row block
-                if (it.partial) fence_proxy_async_smem();
+                // the tensor store or masked bulk copies of the store phase read this row block
+                if (it.partial || (kTma && it.tx >= 0)) fence_proxy_async_smem();
             } else {
                 const int nquads = (it.nload + 3) / 4;   // at most 9: warp 0 takes the ninth
 #pragma unroll
@@ -421,7 +463,12 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
         if (refill) issue(next, st);
 
         const int p = j & 7;
-        if (!kNarrow && mode == kModeShift) {
+        if (kTma && mode == kModeShift && it.tx >= 0) {
+            if (tid == 0) {
+                tma_store_2d(omap, rowblk, it.tx, it.y);
+                bulk_commit();
+            }
+        } else if (!kNarrow && mode == kModeShift) {
             // the 16-byte aligned start of row 0's first chunk; the item owns
             // bytes [lo, hi) of each row's chunk span
             uint8_t *base = scales + (int64_t)it.y * row_stride + it.x - it.lead;
@@ -493,6 +540,22 @@ unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, co
     }
 }
 
+template <bool kDimM, int kWarpsI>
+__global__ void __launch_bounds__(kWarpsI * 32, kWarpsI == 8 ? 3 : 7)
+unrearrange_kernel(const uint8_t *__restrict__ blocked, int64_t blocked_size, const int32_t *__restrict__ ends,
+                   uint8_t *__restrict__ scales, int64_t row_stride, Shape s, int mode) {
+    unrearrange_body<kDimM, kWarpsI, false>(nullptr, 0, blocked, blocked_size, ends, scales, row_stride, s, mode);
+}
+
+// Groups along M in shift mode: items whose owned bytes are one whole box
+// are written with one tensor store each.
+__global__ void __launch_bounds__(kThreads, 3)
+unrearrange_tma_m_kernel(const __grid_constant__ CUtensorMap omap, int64_t map_w, const uint8_t *__restrict__ blocked,
+                         int64_t blocked_size, const int32_t *__restrict__ ends, uint8_t *__restrict__ scales,
+                         int64_t row_stride, Shape s, int mode) {
+    unrearrange_body<true, 8, true>(&omap, map_w, blocked, blocked_size, ends, scales, row_stride, s, mode);
+}
+
 // One warp: the padded start of every group (rows for M, columns for K) and
 // the padded total, as int32[G + 1].
 template <bool kDimM>
@@ -529,15 +592,17 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // how many CTAs of them fit on an SM.
 constexpr int kMaxDevices = 128;
 std::mutex g_inv_mu;
-int g_inv_grid[kMaxDevices][2];   // SMs x resident CTAs (8-warp, narrow instance), 0 until set up
+int g_inv_grid[kMaxDevices][3];   // SMs x resident CTAs: 8-warp, narrow, M tensor-store kernel; 0 until set up
 
-cudaError_t inverse_grid_cap(bool narrow, int *cap) {
+enum InvKernel { kInvWide = 0, kInvNarrow = 1, kInvTmaM = 2 };
+
+cudaError_t inverse_grid_cap(InvKernel which, int *cap) {
     int dev = 0;
     if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_inv_mu);
     if (g_inv_grid[dev][0] == 0) {
-        int sms = 0, occ_m = 0, occ_k = 0, occ_n = 0;
+        int sms = 0, occ_m = 0, occ_k = 0, occ_n = 0, occ_t = 0;
         const cudaError_t steps[] = {
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev),
             cudaFuncSetAttribute(unrearrange_kernel<true, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -546,18 +611,22 @@ cudaError_t inverse_grid_cap(bool narrow, int *cap) {
                                  kInvSmemBytes),
             cudaFuncSetAttribute(unrearrange_kernel<true, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kInvNarrowSmemBytes),
+            cudaFuncSetAttribute(unrearrange_tma_m_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kInvTmaSmemBytes),
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_m, unrearrange_kernel<true, 8>, kThreads, kInvSmemBytes),
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_k, unrearrange_kernel<false, 8>, kThreads, kInvSmemBytes),
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_n, unrearrange_kernel<true, 4>, 128, kInvNarrowSmemBytes),
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_t, unrearrange_tma_m_kernel, kThreads, kInvTmaSmemBytes),
         };
         for (cudaError_t e : steps)
             if (e != cudaSuccess) return e;
         const int occ = occ_m < occ_k ? occ_m : occ_k;
-        if (occ < 1 || occ_n < 1 || sms < 1) return cudaErrorInvalidConfiguration;
-        g_inv_grid[dev][0] = sms * occ;
-        g_inv_grid[dev][1] = sms * occ_n;
+        if (occ < 1 || occ_n < 1 || occ_t < 1 || sms < 1) return cudaErrorInvalidConfiguration;
+        g_inv_grid[dev][kInvWide] = sms * occ;
+        g_inv_grid[dev][kInvNarrow] = sms * occ_n;
+        g_inv_grid[dev][kInvTmaM] = sms * occ_t;
     }
-    *cap = g_inv_grid[dev][narrow ? 1 : 0];
+    *cap = g_inv_grid[dev][which];
     return cudaSuccess;
 }
 
@@ -591,16 +660,35 @@ mx_status unrearrange(mx_group_dim dim, const uint8_t *blocked, int64_t rows, in
                      : (row_stride & 15) == 0                                                  ? kModeShift
                                                                                                 : kModeRows;
     const bool narrow = mode == kModeFlat && s.padded_cols <= kInvNarrowCols;
+    const bool tma_m = mode == kModeShift && dim_m;
     int cap = 0;
-    if (cudaError_t e = inverse_grid_cap(narrow, &cap); e != cudaSuccess) return mx_record_cuda_error(e);
+    if (cudaError_t e = inverse_grid_cap(narrow ? kInvNarrow : tma_m ? kInvTmaM : kInvWide, &cap); e != cudaSuccess)
+        return mx_record_cuda_error(e);
     const int grid = (int)(bound < 1 ? 1 : (bound < cap ? bound : cap));
     const int64_t blocked_size = (int64_t)mx_rearranged_size(dim, rows, cols, G);
-    cudaError_t e = narrow  ? launch_kernel(unrearrange_kernel<true, 4>, grid, 128, kInvNarrowSmemBytes, stream, blocked,
-                                         blocked_size, ends, scales, row_stride, s, mode)
-                    : dim_m ? launch_kernel(unrearrange_kernel<true, 8>, grid, kThreads, kInvSmemBytes, stream, blocked,
-                                         blocked_size, ends, scales, row_stride, s, mode)
-                            : launch_kernel(unrearrange_kernel<false, 8>, grid, kThreads, kInvSmemBytes, stream, blocked,
-                                         blocked_size, ends, scales, row_stride, s, mode);
+    cudaError_t e;
+    if (tma_m) {
+        // Whole-box items go out as tensor stores: a map over the output from
+        // the 16-byte boundary at or below its first byte, as wide as the rows
+        // reach (capped at the row stride; items past the cap use plain stores).
+        CUtensorMap omap;
+        std::memset(&omap, 0, sizeof(omap));
+        const int64_t base_off = (int64_t)(reinterpret_cast<uintptr_t>(scales) & 15u);
+        const int64_t map_w = cols + base_off < row_stride ? cols + base_off : row_stride;
+        if (mx_status st = mx_encode_rows_map(&omap, scales - base_off, map_w, rows, row_stride, 128, 128,
+                                              CU_TENSOR_MAP_SWIZZLE_128B);
+            st != MX_OK)
+            return st;
+        e = launch_kernel(unrearrange_tma_m_kernel, grid, kThreads, kInvTmaSmemBytes, stream, omap, map_w, blocked,
+                          blocked_size, ends, scales, row_stride, s, mode);
+    } else {
+        e = narrow  ? launch_kernel(unrearrange_kernel<true, 4>, grid, 128, kInvNarrowSmemBytes, stream, blocked,
+                                    blocked_size, ends, scales, row_stride, s, mode)
+            : dim_m ? launch_kernel(unrearrange_kernel<true, 8>, grid, kThreads, kInvSmemBytes, stream, blocked,
+                                    blocked_size, ends, scales, row_stride, s, mode)
+                    : launch_kernel(unrearrange_kernel<false, 8>, grid, kThreads, kInvSmemBytes, stream, blocked,
+                                    blocked_size, ends, scales, row_stride, s, mode);
+    }
     return e == cudaSuccess ? MX_OK : mx_record_cuda_error(e);
 }
 

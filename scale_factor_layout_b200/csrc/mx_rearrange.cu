@@ -883,6 +883,27 @@ mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t col
 mx_status mx_record_cuda_error(cudaError_t e) { return mx::cuda_status(e); }
 cudaError_t mx_inverse_flags(unsigned int *flags, int clear);   // defined in mx_inverse.cu
 
+// A 2-D uint8 tensor map over `rows` rows of `width` bytes at `row_stride`
+// (a multiple of 16) from the 16-byte aligned `base`, boxes of box_w x box_h
+// with the given swizzle, for the current device (whose primary context is
+// made current in this thread first, as the encoder needs).
+mx_status mx_encode_rows_map(CUtensorMap *map, const void *base, int64_t width, int64_t rows, int64_t row_stride,
+                             uint32_t box_w, uint32_t box_h, CUtensorMapSwizzle swizzle) {
+    const mx::DeviceInfo *d = nullptr;
+    if (mx_status st = mx::device_info(&d); st != MX_OK) return st;
+    auto encode = mx::encode_fn();
+    if (encode == nullptr) return mx::cuda_status(cudaErrorSymbolNotFound);
+    cuuint64_t gdim[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+    cuuint64_t gstride[1] = {(cuuint64_t)row_stride};
+    cuuint32_t box[2] = {box_w, box_h};
+    cuuint32_t estride[2] = {1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), gdim, gstride, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return mx::cuda_status(static_cast<cudaError_t>(r));   // driver code
+    return MX_OK;
+}
+
 // ------------------------------------------------------------------ C ABI
 extern "C" {
 
