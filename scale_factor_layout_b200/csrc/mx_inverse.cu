@@ -277,10 +277,15 @@ constexpr int kModeFlat = 2;    // rows back to back (stride == cols <= 128)
 //     l % 8 of row l / 8 (one 128-bit store covers four contiguous runs), a
 //     ninth chunk by the row's first lane.  Shift mode: whole chunks are
 //     plain stores, partial ones (where a run starts or ends) masked bulk
-//     copies.  Rows mode: each chunk is shifted into place from the 32-byte
-//     window around it, partial ones stored by words and bytes.  Flat mode
-//     (rows back to back in memory): the item's rows are one contiguous span
-//     and threads take its chunks in order.
+//     copies; with kTma (groups along M), an item that owns exactly one
+//     128 x 128-byte box had its row block written 128B-swizzled in step 1
+//     and thread 0 writes it with one tensor store.  Rows mode: each chunk is
+//     shifted into place from the 32-byte window around it, partial ones
+//     stored by words and bytes.  Flat mode (rows back to back in memory):
+//     the item's rows are one contiguous span and threads take its chunks in
+//     order.
+// The kernels below instantiate this body: unrearrange_kernel for every mode
+// without tensor stores, unrearrange_tma_m_kernel for shift mode along M.
 template <bool kDimM, int kWarpsI, bool kTma>
 __device__ __forceinline__ void unrearrange_body(const CUtensorMap *omap, int64_t map_w,
                                                  const uint8_t *__restrict__ blocked, int64_t blocked_size,
