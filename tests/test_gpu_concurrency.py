@@ -66,3 +66,33 @@ def test_fresh_thread_legacy_stream(mxlib, orc):
     for dc in dcs:
         c = dc.case
         assert np.array_equal(dc.output(), orc.rearrange(c.dim, c.scales, c.ends)), c.name
+
+
+def test_fresh_thread_inverse(mxlib, orc):
+    """The inverse from a host thread whose first CUDA work is the library call
+    (the M-groups path encodes an output tensor map, a driver call that needs
+    the device's context current in that thread)."""
+    cases = [synth.m_wide(), synth.k_groups(), synth.m_skinny()]
+    prepared = []
+    for c in cases:
+        blocked_np = orc.rearrange(c.dim, c.scales, c.ends)
+        blocked = torch.from_numpy(blocked_np).cuda()
+        ends = torch.from_numpy(np.ascontiguousarray(c.ends, dtype=np.int32)).cuda()
+        out = torch.full((c.rows, c.cols), 0xEE, dtype=torch.uint8, device="cuda")
+        prepared.append((c, blocked_np, blocked, ends, out))
+    torch.cuda.synchronize()
+    results = []
+
+    def worker(c, blocked, ends, out):
+        fn = B.mx_unrearrange_m_groups if c.dim == synth.DIM_M else B.mx_unrearrange_k_groups
+        st = fn(blocked.data_ptr(), c.rows, c.cols, ends.data_ptr(), len(c.ends), out.data_ptr(), c.cols, 0)
+        results.append((c.name, st, B.mx_last_cuda_error()))
+
+    for c, _, blocked, ends, out in prepared:
+        t = threading.Thread(target=worker, args=(c, blocked, ends, out))
+        t.start()
+        t.join(60)
+    assert all(st == B.MX_OK for _, st, _ in results), results
+    torch.cuda.synchronize()
+    for c, blocked_np, _, _, out in prepared:
+        assert np.array_equal(out.cpu().numpy(), orc.inverse(c.dim, blocked_np, c.rows, c.cols, c.ends)), c.name
