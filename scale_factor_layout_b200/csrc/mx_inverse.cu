@@ -73,7 +73,7 @@ constexpr int kInvTmaSmemBytes = kInvStages * kInvStageBytes + 2 * kInvBlockByte
 // (1032 row blocks of a 131072-row input, 1036 CTAs on a B200).
 constexpr int kInvNarrowCols = 48;
 constexpr int kInvNarrowStageBytes = (kInvNarrowCols / 4) * 512;             // 6 KB
-constexpr int kInvNarrowBlockBytes = kTileRows * kInvNarrowCols;             // 6 KB
+constexpr int kInvNarrowBlockBytes = kTileRows * kInvNarrowCols + 16;        // 6 KB and a chunk's offset
 constexpr int kInvNarrowSmemBytes = kInvStages * kInvNarrowStageBytes + 2 * kInvNarrowBlockBytes + 128;
 constexpr uint32_t kInvFlagWaitTimeout = 1u;
 
@@ -257,7 +257,7 @@ __device__ __forceinline__ void store_chunk_shift(uint8_t *row, const uint8_t *s
 
 constexpr int kModeRows = 0;    // rows start at different offsets within a 16-byte chunk
 constexpr int kModeShift = 1;   // row stride a multiple of 16: one offset for all rows of an item
-constexpr int kModeFlat = 2;    // rows back to back (stride == cols <= 128)
+constexpr int kModeFlat = 2;    // rows back to back (stride == cols <= 128), output 4-byte aligned
 
 // Persistent CTAs walk work items round-robin; one thread streams each item's
 // tiles (one contiguous, 512-byte aligned span of the blocked buffer) into a
@@ -293,7 +293,6 @@ __device__ __forceinline__ void unrearrange_body(const CUtensorMap *omap, int64_
                                                  int64_t row_stride, const Shape &s, int mode) {
     static_assert(kWarpsI == 8 || kWarpsI == 4, "8 warps (every mode) or 4 (narrow flat rows)");
     constexpr bool kNarrow = kWarpsI == 4;
-    constexpr int kThr = kWarpsI * 32;
     constexpr int kStageB = kNarrow ? kInvNarrowStageBytes : kInvStageBytes;
     constexpr int kBlockB = kNarrow ? kInvNarrowBlockBytes : kInvBlockBytes;
     constexpr int kPasses = kNarrow ? 1 : 2;   // quads of tiles per thread (at most 3, or 9)
@@ -305,7 +304,7 @@ __device__ __forceinline__ void unrearrange_body(const CUtensorMap *omap, int64_
     uint8_t *rowblks = stages + kInvStages * kStageB;
     __shared__ GroupTable table;
     __shared__ __align__(8) uint64_t full[kInvStages];
-    __shared__ InvItem items[kInvStages];
+    __shared__ InvItem items[kInvStages + 1];   // [kInvStages]: the next refill, decoded ahead
     const int tid = threadIdx.x;
     const int j = tid & 31;
     const int q = tid >> 5;
@@ -352,10 +351,10 @@ __device__ __forceinline__ void unrearrange_body(const CUtensorMap *omap, int64_
     for (int n = 0; n < n_my; ++n) {
         const int st = n % kInvStages;
         // The refill of this stage is decoded while its current copy is in
-        // flight, so that only the copy itself is issued after the barrier.
+        // flight, so that only the copy itself is issued after the barrier; it
+        // waits in shared memory, not in registers held through the transpose.
         const bool refill = tid == 0 && n + kInvStages < n_my;
-        InvItem next;
-        if (refill) next = decode(n + kInvStages);
+        if (refill) items[kInvStages] = decode(n + kInvStages);
         const bool ok = mbar_wait_bounded(&full[st], (uint32_t)(n / kInvStages) & 1u);
         InvItem it;
         uint8_t *rowblk = rowblks + (n & 1) * kBlockB;
@@ -441,15 +440,23 @@ __device__ __forceinline__ void unrearrange_body(const CUtensorMap *omap, int64_
                         if (!kNarrow && mode == kModeRows) {
                             *reinterpret_cast<uint4 *>(rowblk + r * kInvPitch + 16 * qq) =
                                 make_uint4(word_of(w[0], a), word_of(w[1], a), word_of(w[2], a), word_of(w[3], a));
-                        } else {
-                            // rows back to back: word-aligned (cols is a multiple of 4), stop at the row's end
-                            uint32_t *dst = reinterpret_cast<uint32_t *>(rowblk + r * s.cols) + 4 * qq;
+                        } else if (kDimM) {
+                            // Flat mode: the item's rows go to the row block as one span that
+                            // starts `flead` bytes in (its offset within a 16-byte chunk of the
+                            // output, a multiple of 4), so that its output chunks sit 16-byte
+                            // aligned; word stores (cols is a multiple of 4), stopping at the
+                            // row's end.
+                            const int flead =
+                                (int)((reinterpret_cast<uintptr_t>(scales) + (uint64_t)it.y * s.cols) & 15u);
+                            uint32_t *dst = reinterpret_cast<uint32_t *>(rowblk + flead + r * s.cols) + 4 * qq;
 #pragma unroll
                             for (int t = 0; t < 4; ++t)
                                 if (16 * qq + 4 * t < s.cols) dst[t] = word_of(w[t], a);
                         }
                     }
                 }
+                // the bulk copies of the store phase read this row block
+                if (kDimM && mode == kModeFlat) fence_proxy_async_smem();
             }
         }
         // this thread's masked copies of item n - 1 have read their row block,
@@ -465,7 +472,7 @@ __device__ __forceinline__ void unrearrange_body(const CUtensorMap *omap, int64_
             }
             return;
         }
-        if (refill) issue(next, st);
+        if (refill) issue(items[kInvStages], st);
 
         const int p = j & 7;
         if (kTma && mode == kModeShift && it.tx >= 0) {
@@ -514,16 +521,22 @@ __device__ __forceinline__ void unrearrange_body(const CUtensorMap *omap, int64_
                         store16_part(row + c8, window16(src, c8 + it.pre, kInvPitch), 0, min(16, hi_own - c8));
                 }
             }
-        } else {
+        } else if (kDimM && tid == 0) {
+            // Flat mode (groups along M only): the item's output is one span, `lead` bytes into a 16-byte
+            // chunk, at the same offset in the row block: whole chunks go out as
+            // one bulk copy, a partial first and last chunk as masked copies.
             const int span = it.rows_valid * s.cols;
-            uint8_t *base = scales + (int64_t)it.y * s.cols;   // the item's first byte
-            const int lead = (int)(reinterpret_cast<uintptr_t>(base) & 15u);
-            const int nch = (lead + span + 15) >> 4;
-            for (int c = tid; c < nch; c += kThr) {
-                const int o = 16 * c - lead;
-                const int kmin = max(0, -o), kmax = min(16, span - o);
-                store16_part(base + o, window16(rowblk, o, kBlockB), kmin, kmax);
-            }
+            uint8_t *chunk0 = scales + (int64_t)it.y * s.cols;   // the item's first byte ...
+            const int lead = (int)(reinterpret_cast<uintptr_t>(chunk0) & 15u);
+            chunk0 -= lead;                                      // ... and its chunk's start
+            const int end = lead + span;
+            const int kf0 = lead ? 1 : 0, kf1 = end >> 4;        // whole chunks [kf0, kf1)
+            if (kf1 > kf0) bulk_store_s2g(chunk0 + 16 * kf0, rowblk + 16 * kf0, (uint32_t)(kf1 - kf0) * 16u);
+            if (lead)
+                bulk_store16_masked(chunk0, rowblk, (uint16_t)(((1u << min(16, end)) - 1u) & ~((1u << lead) - 1u)));
+            if ((end & 15) && (kf1 > 0 || !lead))
+                bulk_store16_masked(chunk0 + 16 * kf1, rowblk + 16 * kf1, (uint16_t)((1u << (end & 15)) - 1u));
+            bulk_commit();
         }
     }
     // the masked copies read shared memory, which must outlive them
@@ -661,7 +674,9 @@ mx_status unrearrange(mx_group_dim dim, const uint8_t *blocked, int64_t rows, in
                                 : ceil_div(rows, 128) * (ceil_div(cols, kChunkCols) + G);
     if (bound > INT_MAX) return MX_ERR_UNSUPPORTED;
     // flat mode: rows back to back, one item per row block, whole words
-    const int mode = dim_m && row_stride == cols && cols <= kTilesPerChunk * 4 && cols % 4 == 0 ? kModeFlat
+    const int mode = dim_m && row_stride == cols && cols <= kTilesPerChunk * 4 && cols % 4 == 0 &&
+                             (reinterpret_cast<uintptr_t>(scales) & 3u) == 0
+                         ? kModeFlat
                      : (row_stride & 15) == 0                                                  ? kModeShift
                                                                                                 : kModeRows;
     const bool narrow = mode == kModeFlat && s.padded_cols <= kInvNarrowCols;
