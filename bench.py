@@ -144,14 +144,14 @@ def kernel_source_sha(root: str = ROOT, op: str = "rearrange") -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(call: str, op: str = "rearrange"):
+def ncu_traffic(call: str, op: str = "rearrange", root: str = ROOT, path: str | None = None):
     """DRAM bytes per launch recorded by an ncu capture (profiles/ncu_traffic.txt)
     of the op's kernel for this call, or None when absent or taken on different
     kernel sources."""
-    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    path = path or os.path.join(root, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
-    sha = kernel_source_sha(op=op)
+    sha = kernel_source_sha(root, op=op)
     for line in open(path):
         if line.startswith("#") or not line.strip():
             continue

@@ -1,0 +1,60 @@
+"""Host-side helpers of bench.py: the device-code key that ties the DRAM
+traffic figures of profiles/ncu_traffic.txt to the kernels they were taken on."""
+import os
+import shutil
+
+import bench
+
+
+def _copy_tree(tmp_path):
+    dst = tmp_path / "scale_factor_layout_b200" / "csrc"
+    dst.mkdir(parents=True)
+    src = os.path.join(bench.ROOT, "scale_factor_layout_b200", "csrc")
+    for name in ("mx_device.cuh", "mx_rearrange.cu", "mx_inverse.cu"):
+        shutil.copy(os.path.join(src, name), dst / name)
+    return dst
+
+
+def _keys(root):
+    return bench.kernel_source_sha(root), bench.kernel_source_sha(root, op="inverse")
+
+
+def test_key_ignores_comments_and_host_code(tmp_path):
+    csrc = _copy_tree(tmp_path)
+    before = _keys(str(tmp_path))
+    p = csrc / "mx_device.cuh"
+    p.write_text(p.read_text().replace("namespace mx {", "namespace mx {\n// a comment added\n\n", 1))
+    for name in ("mx_rearrange.cu", "mx_inverse.cu"):
+        q = csrc / name
+        q.write_text(q.read_text() + "\nstatic int host_side_addition = 0;\n")
+    assert _keys(str(tmp_path)) == before
+
+
+def test_key_tracks_each_ops_device_code(tmp_path):
+    csrc = _copy_tree(tmp_path)
+    fwd, inv = _keys(str(tmp_path))
+    q = csrc / "mx_inverse.cu"
+    text = q.read_text()
+    cut = text.index(bench.HOST_MARKER.decode())
+    assert "kInvStages = 2" in text[:cut]
+    q.write_text(text[:cut].replace("kInvStages = 2", "kInvStages = 3", 1) + text[cut:])
+    assert bench.kernel_source_sha(str(tmp_path)) == fwd
+    assert bench.kernel_source_sha(str(tmp_path), op="inverse") != inv
+    p = csrc / "mx_device.cuh"     # shared by both ops
+    p.write_text(p.read_text().replace("constexpr int kTileRows = 128;", "constexpr int kTileRows = 256;", 1))
+    assert bench.kernel_source_sha(str(tmp_path)) != fwd
+
+
+def test_traffic_lookup_by_op_call_and_key(tmp_path):
+    _copy_tree(tmp_path)
+    fwd, inv = _keys(str(tmp_path))
+    traffic = tmp_path / "traffic.txt"
+    traffic.write_text("# header\n"
+                       f"op=rearrange call=k_groups bytes_per_launch=111 source_sha={fwd} capture=a.md\n"
+                       f"op=inverse call=k_groups bytes_per_launch=222 source_sha={inv} capture=b.md\n"
+                       f"op=inverse call=m_wide bytes_per_launch=333 source_sha=0000000000000000 capture=c.md\n")
+    root, path = str(tmp_path), str(traffic)
+    assert bench.ncu_traffic("k_groups", "rearrange", root, path) == 111
+    assert bench.ncu_traffic("k_groups", "inverse", root, path) == 222
+    assert bench.ncu_traffic("m_wide", "inverse", root, path) is None      # taken on other kernels
+    assert bench.ncu_traffic("m_skinny", "rearrange", root, path) is None  # never captured
