@@ -459,8 +459,9 @@ __device__ __forceinline__ void unrearrange_body(const CUtensorMap *omap, int64_
                 if (kDimM && mode == kModeFlat) fence_proxy_async_smem();
             }
         }
-        // this thread's masked copies of item n - 1 have read their row block,
-        // which item n + 1 overwrites after the barrier
+        // this thread's bulk copies of item n - 1 (masked chunks, a tensor store,
+        // a flat span) have read their row block, which item n + 1 overwrites
+        // after the barrier
         bulk_wait_read<0>();
         if (__syncthreads_or(!ok)) {
             // A copy never completed: flag it, wait (bounded) for the copies
@@ -522,9 +523,10 @@ __device__ __forceinline__ void unrearrange_body(const CUtensorMap *omap, int64_
                 }
             }
         } else if (kDimM && tid == 0) {
-            // Flat mode (groups along M only): the item's output is one span, `lead` bytes into a 16-byte
-            // chunk, at the same offset in the row block: whole chunks go out as
-            // one bulk copy, a partial first and last chunk as masked copies.
+            // Flat mode (groups along M only): the item's output is one span,
+            // `lead` bytes into a 16-byte chunk, at the same offset in the row
+            // block: whole chunks go out as one bulk copy, a partial first and
+            // last chunk as masked copies.
             const int span = it.rows_valid * s.cols;
             uint8_t *chunk0 = scales + (int64_t)it.y * s.cols;   // the item's first byte ...
             const int lead = (int)(reinterpret_cast<uintptr_t>(chunk0) & 15u);
@@ -539,7 +541,7 @@ __device__ __forceinline__ void unrearrange_body(const CUtensorMap *omap, int64_
             bulk_commit();
         }
     }
-    // the masked copies read shared memory, which must outlive them
+    // the bulk copies read shared memory, which must outlive them
     bulk_wait_all();
 
     // Elements no group covers (rows past the last end for M, columns past
