@@ -119,3 +119,45 @@ def test_torch_wrappers_reject_bad_tensors():
         mxs.unrearrange(mxs.MX_GROUPS_M, torch.zeros(4096, dtype=torch.uint8), 20, 8, ends)
     with pytest.raises(ValueError):   # offsets of the wrong dtype
         mxs.padded_group_starts(mxs.MX_GROUPS_M, 20, 8, torch.tensor([10, 20], dtype=torch.int64))
+
+
+def test_header_is_plain_c_and_links(mxlib, tmp_path):
+    """include/mxscale.h compiles as C (not C++), every declared entry point
+    links against libmxscale.so, and the host-only calls run from C."""
+    import os
+    import shutil
+    import subprocess
+
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    names = B.declared_symbols()
+    refs = "\n".join(f"    (entry_fn)&{n}," for n in names)
+    src = tmp_path / "use_mxscale.c"
+    src.write_text(f'''#include <stdio.h>
+#include "mxscale.h"
+typedef void (*entry_fn)(void);
+static const entry_fn entry_points[] = {{
+{refs}
+}};
+int main(void) {{
+    size_t n = sizeof entry_points / sizeof entry_points[0];
+    for (size_t i = 0; i < n; ++i)
+        if (entry_points[i] == 0) return 2;
+    printf("%zu %d %zu %zu %s\\n", n, mx_version(),
+           mx_rearranged_size(MX_GROUPS_M, 1000, 44, 4), mx_rearranged_size(MX_GROUPS_K, 7168, 4096, 8),
+           mx_status_string(MX_ERR_MISALIGNED));
+    return 0;
+}}
+''')
+    exe = tmp_path / "use_mxscale"
+    lib_dir = os.path.dirname(B.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-pedantic", "-I", os.path.dirname(B.HEADER),
+                    "-I", cuda_inc, str(src), "-o", str(exe), "-L", lib_dir, "-lmxscale",
+                    f"-Wl,-rpath,{lib_dir}"], check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split(maxsplit=4)
+    assert int(out[0]) == len(names)
+    assert int(out[1]) == B.mx_version()
+    assert int(out[2]) == B.mx_rearranged_size(M, 1000, 44, 4)
+    assert int(out[3]) == B.mx_rearranged_size(K, 7168, 4096, 8)
+    assert out[4].strip() == B.status_string(B.MX_ERR_MISALIGNED)
