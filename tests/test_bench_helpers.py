@@ -58,3 +58,18 @@ def test_traffic_lookup_by_op_call_and_key(tmp_path):
     assert bench.ncu_traffic("k_groups", "inverse", root, path) == 222
     assert bench.ncu_traffic("m_wide", "inverse", root, path) is None      # taken on other kernels
     assert bench.ncu_traffic("m_skinny", "rearrange", root, path) is None  # never captured
+
+
+def test_algorithmic_bytes_match_the_oracle(orc):
+    """The bytes behind the bench's GB/s (real input read, exact padded output
+    written, the allocation) agree with the oracle's own counts."""
+    from scale_factor_layout_b200 import synth
+
+    cases = [f() for f in synth.NAMED.values()]
+    cases += [synth.k_sweep_point(i, k) for i in (0, 3, 6) for k in (0, 5, 9)]
+    cases += [synth.random_small(seed) for seed in range(900, 1100)]
+    for c in cases:
+        b = bench.algorithmic_bytes(c)
+        assert b["read"] == orc.read_bytes(c.dim, c.rows, c.cols, c.ends), c.name
+        assert b["written"] == orc.written_bytes(c.dim, c.rows, c.cols, c.ends), c.name
+        assert b["alloc"] == orc.rearranged_size(c.dim, c.rows, c.cols, len(c.ends)), c.name
