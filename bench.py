@@ -10,12 +10,18 @@ Metric: GB/s = (bytes of real scales read + exact padded bytes written) / time,
 and the same as a fraction of the measured HBM copy bandwidth.
 
 Timing: the K timed steps are captured in one CUDA graph (as the pages timed
-their kernels) and replayed once between two CUDA events; inputs and outputs
-rotate over enough buffer sets that one rotation spans more than 4x the L2,
-so every step reads cold inputs.  Each call's own duration comes from a
-second graph per call type: the same K launches of that call, back to back,
-between two CUDA events.  Multi-GPU: independent replicas, one process per
-GPU (torchrun), max time over ranks.
+their kernels), uploaded to the device, and replayed once between two CUDA
+events right after the warm-up graph; inputs and outputs rotate over enough
+buffer sets that one rotation spans more than 4x the L2, so every step reads
+cold inputs.  Each call's own per-launch duration (the roofline figure) comes
+from a graph of that call's launches alone, back to back over the same
+rotation, at least --call-launches of them so that the figure is the steady
+state whatever K is: one untimed replay, then one timed replay.
+Multi-GPU: independent replicas, one process per GPU (torchrun), max time
+over ranks.
+
+--workload k_sweep times every point of the K-groups sweep (M x TotalK, 70
+points) the same way, each beside a same-size device copy and the CPU oracle.
 
 --impl reference times the CPU oracle (the plain C statement of the layout)
 on this host on a bounded sample of the same workload.
@@ -51,6 +57,7 @@ WORKLOAD_DESC = {
     "k_groups": "K-groups 7168x4096 G=8 (TMA)",
 }
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, nominal (the measured copy peak is the roofline's denominator)
 L2_BYTES = 126 * 2**20
 METRIC = "rearrange GB/s (read+padded write) and % of B200 HBM peak, 1 GPU"
 
@@ -83,6 +90,8 @@ def algorithmic_bytes(case) -> dict:
 def make_cases(workload: str):
     from scale_factor_layout_b200 import synth
 
+    if workload == "k_sweep":
+        return [synth.k_sweep_point(i, k) for i, k in synth.sweep_points()]
     if workload.startswith("k_sweep_"):
         m, total_k = (int(v) for v in workload[len("k_sweep_"):].split("x"))
         return [synth.k_sweep_point(synth.SWEEP_ROWS.index(m), synth.SWEEP_TOTAL_K.index(total_k))]
@@ -90,6 +99,8 @@ def make_cases(workload: str):
 
 
 def workload_desc(workload: str) -> str:
+    if workload == "k_sweep":
+        return "K-groups sweep: M in {128..28672} x TotalK in {2^10..2^19}, scales M x TotalK/32, G=8 (70 points)"
     if workload.startswith("k_sweep_"):
         m, total_k = (int(v) for v in workload[len("k_sweep_"):].split("x"))
         return f"K-groups sweep point M={m} TotalK={total_k}: scales {m}x{total_k // 32}, G=8 (TMA)"
@@ -99,7 +110,7 @@ def workload_desc(workload: str) -> str:
 def workload_arg(value: str) -> str:
     from scale_factor_layout_b200 import synth
 
-    if value in WORKLOADS:
+    if value in WORKLOADS or value == "k_sweep":
         return value
     if value.startswith("k_sweep_"):
         try:
@@ -144,10 +155,12 @@ def kernel_source_sha(root: str = ROOT, op: str = "rearrange") -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(call: str, op: str = "rearrange", root: str = ROOT, path: str | None = None):
+def ncu_traffic(call: str, op: str = "rearrange", root: str = ROOT, path: str | None = None,
+                detail: bool = False):
     """DRAM bytes per launch recorded by an ncu capture (profiles/ncu_traffic.txt)
     of the op's kernel for this call, or None when absent or taken on different
-    kernel sources."""
+    kernel sources.  With detail=True: {"read", "write", "l2_write"} (l2_write,
+    the bytes the kernel wrote into L2, is None where the capture lacks it)."""
     path = path or os.path.join(root, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -157,7 +170,11 @@ def ncu_traffic(call: str, op: str = "rearrange", root: str = ROOT, path: str | 
             continue
         kv = dict(tok.split("=", 1) for tok in line.split() if "=" in tok)
         if kv.get("op", "rearrange") == op and kv.get("call") == call and kv.get("source_sha") == sha:
-            return int(float(kv["bytes_per_launch"]))
+            if not detail:
+                return int(float(kv["bytes_per_launch"]))
+            l2w = kv.get("l2_write")
+            return {"read": int(float(kv["read"])), "write": int(float(kv["write"])),
+                    "l2_write": int(float(l2w)) if l2w is not None else None}
     return None
 
 
@@ -311,6 +328,106 @@ def launch(item, stream_handle, op="rearrange", path="auto"):
         raise RuntimeError(f"{c.name}: {B.status_string(st)}")
 
 
+_libcuda = None
+
+
+def upload_graph(g, stream_handle: int) -> None:
+    """Upload a captured graph's executable to the device ahead of its first
+    replay (cuGraphUpload), so that no timed replay pays for the upload."""
+    global _libcuda
+    import ctypes
+
+    if _libcuda is None:
+        lib = ctypes.CDLL("libcuda.so.1")
+        lib.cuGraphUpload.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+        lib.cuGraphUpload.restype = ctypes.c_int
+        _libcuda = lib
+    r = _libcuda.cuGraphUpload(ctypes.c_void_p(g.raw_cuda_graph_exec()), ctypes.c_void_p(stream_handle))
+    if r != 0:
+        raise RuntimeError(f"cuGraphUpload failed (CUresult {r})")
+
+
+class GraphTimer:
+    """CUDA graphs of launches on one stream, timed with CUDA events on that
+    stream, barrier and synchronize on both sides, max over ranks."""
+
+    def __init__(self, stream, dist, device):
+        self.stream, self.dist, self.device = stream, dist, device
+        self.handle = stream.cuda_stream
+
+    def capture(self, fn_calls):
+        """One graph holding the calls (each a zero-argument callable that
+        enqueues work on the stream), uploaded to the device."""
+        import torch
+
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(self.stream):
+            with torch.cuda.graph(g, stream=self.stream):
+                for fn in fn_calls:
+                    fn()
+        upload_graph(g, self.handle)
+        return g
+
+    def replay(self, g):
+        import torch
+
+        with torch.cuda.stream(self.stream):
+            g.replay()
+
+    def time(self, g, pre=None) -> float:
+        """Seconds of one replay of g (max over ranks); `pre` is replayed
+        untimed right before, on the same stream."""
+        import torch
+
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier(self.dist, self.device)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(self.stream):
+            if pre is not None:
+                pre.replay()
+            start.record(self.stream)
+            g.replay()
+            end.record(self.stream)
+        torch.cuda.synchronize()
+        barrier(self.dist, self.device)
+        return max_over_ranks(start.elapsed_time(end) / 1e3, self.dist, self.device)
+
+    def steady(self, g, n: int) -> float:
+        """Average seconds per launch of a graph of n launches back to back:
+        one untimed replay, then one timed replay."""
+        self.replay(g)
+        return self.time(g) / n
+
+
+def per_launch_launches(steps: int, minimum: int) -> int:
+    """Launches in each per-call timing graph: the timed step count, but at
+    least `minimum`, so that the per-launch figure is the steady state of
+    back-to-back launches whatever --steps is."""
+    return max(steps, minimum)
+
+
+def roofline_entry(kernel: str, case_name: str, bytes_moved: int, seconds: float, peak: float, peak_src: str,
+                   traffic) -> dict:
+    """The roofline object of the bench line for the dominant kernel."""
+    achieved = bytes_moved / seconds / 1e9
+    out = {"bound": "hbm", "kernel": f"{kernel} ({case_name})", "achieved": round(achieved, 1), "peak": peak,
+           "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} hbm_gbs",
+           "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+           "algorithmic_bytes": bytes_moved, "traffic": None}
+    if traffic is not None:
+        out["traffic"] = traffic["read"] + traffic["write"]
+        out["traffic_read"] = traffic["read"]
+        out["traffic_write"] = traffic["write"]
+        if traffic.get("l2_write") is not None:
+            out["traffic_l2_write"] = traffic["l2_write"]
+        if traffic["write"] < 0.1 * (bytes_moved - traffic["read"]):
+            out["traffic_note"] = ("read-dominated: the launch's output is still in L2 when it ends (written back "
+                                   "to DRAM later); traffic_l2_write is what the kernel wrote to L2")
+    return out
+
+
 def run_ours(args, rank, world, local):
     import torch
 
@@ -322,6 +439,8 @@ def run_ours(args, rank, world, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     dist = dist_init(world, "nccl")
+    if args.workload == "k_sweep":
+        return run_sweep(args, rank, world, device, dist)
     cases = make_cases(args.workload)
     per_call = [algorithmic_bytes(c) for c in cases]
     step_bytes = sum(b["read"] + b["written"] for b in per_call)
@@ -333,6 +452,7 @@ def run_ours(args, rank, world, local):
     stream = torch.cuda.Stream(device)
     h = stream.cuda_stream
     ncalls = len(cases)
+    timer = GraphTimer(stream, dist, device)
 
     def step_items(k):
         return [r[k % len(r)] for r in rot]
@@ -343,87 +463,64 @@ def run_ours(args, rank, world, local):
                 launch(it, h, args.op, args.path)
     torch.cuda.synchronize()
 
-    def capture(launches):
-        """One CUDA graph holding the given (item) launches back to back."""
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(stream):
-            with torch.cuda.graph(g, stream=stream):
-                for it in launches:
-                    launch(it, h, args.op, args.path)
-        return g
+    def calls_of(items):
+        return [lambda it=it: launch(it, h, args.op, args.path) for it in items]
 
     def steps_of(k0, n):
         return [it for k in range(k0, k0 + n) for it in step_items(k)]
 
-    def replay_timed(g):
-        start = torch.cuda.Event(enable_timing=True)
-        end = torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        barrier(dist, device)
-        torch.cuda.synchronize()
-        with torch.cuda.stream(stream):
-            start.record(stream)
-            g.replay()
-            end.record(stream)
-        torch.cuda.synchronize()
-        barrier(dist, device)
-        return start.elapsed_time(end) / 1e3
-
-    def capture_copies(i):
+    def copies_of(i, n):
         """The practical ceiling for call i: a D2D copy of its input bytes
         (read + write the same traffic), same rotation, same graph timing."""
         srcs = [it[1] for it in rot[i]]
         dsts = [torch.empty_like(x) for x in srcs]
-        g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
             for a, b in zip(srcs, dsts):   # warm the copy path outside capture
                 b.copy_(a)
-            torch.cuda.synchronize()
-            with torch.cuda.graph(g, stream=stream):
-                for k in range(args.steps):
-                    dsts[k % len(dsts)].copy_(srcs[k % len(srcs)])
-        return g, dsts
+        torch.cuda.synchronize()
+        return [lambda a=srcs[k % len(srcs)], b=dsts[k % len(dsts)]: b.copy_(a) for k in range(n)], dsts
 
-    warm_g = capture(steps_of(0, args.warmup))
-    timed_g = capture(steps_of(args.warmup, args.steps))
-    # each call on its own: the same launches back to back, one call type per graph
-    per_call_g = [capture([rot[i][k % len(rot[i])] for k in range(args.steps)]) for i in range(ncalls)]
-    copy_g = [capture_copies(i) for i in range(ncalls)] if not args.no_copy_ceiling else None
+    warm_g = timer.capture(calls_of(steps_of(0, args.warmup)))
+    timed_g = timer.capture(calls_of(steps_of(args.warmup, args.steps)))
 
     sampler = ClockSampler(local)
     with sampler:
-        with torch.cuda.stream(stream):
-            warm_g.replay()
+        timer.replay(warm_g)
         t0 = time.perf_counter()
-        seconds = replay_timed(timed_g)
+        seconds_max = timer.time(timed_g)
         t1 = time.perf_counter()
         sampler.window = (t0, t1)
-        avg = []
-        for g in per_call_g:
-            with torch.cuda.stream(stream):
-                warm_g.replay()
-            avg.append(max_over_ranks(replay_timed(g), dist, device) / args.steps)
-        copy_avg = None
-        if copy_g is not None:
+        del timed_g
+        # Each call's own per-launch duration: its launches back to back in a
+        # graph of their own (same rotation, cold inputs), in steady state.
+        n_call = per_launch_launches(args.steps, args.call_launches)
+        avg, copy_avg = [], None
+        for i in range(ncalls):
+            g = timer.capture(calls_of([rot[i][k % len(rot[i])] for k in range(n_call)]))
+            avg.append(timer.steady(g, n_call))
+            del g
+        if not args.no_copy_ceiling:
             copy_avg = []
-            for g, _ in copy_g:
-                with torch.cuda.stream(stream):
-                    warm_g.replay()
-                copy_avg.append(max_over_ranks(replay_timed(g), dist, device) / args.steps)
-    seconds_max = max_over_ranks(seconds, dist, device)
-    del timed_g, warm_g, per_call_g, copy_g
+            for i in range(ncalls):
+                fns, dsts = copies_of(i, n_call)
+                g = timer.capture(fns)
+                copy_avg.append(timer.steady(g, n_call))
+                del g, dsts
+    del warm_g
 
     peak, peak_src = load_peaks()
     value = aggregate_value(step_bytes, args.steps, world, seconds_max)
     calls = []
     for ci, (c, b, t) in enumerate(zip(cases, per_call, avg)):
         gbs = (b["read"] + b["written"]) / t / 1e9
-        path = (mxs.mx_select_path(c.dim, rot[cases.index(c)][0][1].data_ptr(), c.rows, c.cols, c.cols)
+        path = (mxs.mx_select_path(c.dim, rot[ci][0][1].data_ptr(), c.rows, c.cols, c.cols)
                 if args.path == "auto" else B.PATHS[args.path])
         calls.append({"case": c.name, "path": B.PATH_NAMES.get(path, "?"),
                       "us": round(t * 1e6, 3), "gbps": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
+                      "frac_of_nominal": round(gbs / NOMINAL_HBM_GBS, 4),
                       "read_bytes": b["read"], "written_bytes": b["written"], "alloc_bytes": b["alloc"],
-                      "gbps_pages_convention": round((b["read"] + b["alloc"]) / t / 1e9, 1)})
+                      "gbps_pages_convention": round((b["read"] + b["alloc"]) / t / 1e9, 1),
+                      "launches_timed": n_call})
         if copy_avg is not None:
             cbytes = 2 * c.rows * c.cols   # the copy reads and writes the input's bytes
             cg = cbytes / copy_avg[ci] / 1e9
@@ -431,15 +528,12 @@ def run_ours(args, rank, world, local):
                               "frac_of_copy": round(gbs / cg, 4)})
     dom = max(range(ncalls), key=lambda i: avg[i])
     dc = calls[dom]
-    achieved = dc["read_bytes"] + dc["written_bytes"]
     kernel_names = {"tma": "rearrange_tma_m" if cases[dom].dim == 0 else "rearrange_tma_k",
                     "flat": "rearrange_flat_tma", "word": "rearrange_fallback", "byte": "rearrange_fallback"}
     kname = "unrearrange_kernel" if args.op == "inverse" else kernel_names.get(dc["path"], "?")
-    roofline = {"bound": "hbm", "kernel": f"{kname} ({dc['case']})",
-                "achieved": round(achieved / avg[dom] / 1e9, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / avg[dom] / 1e9 / peak, 4), "peak_source": f"{peak_src} hbm_gbs",
-                "traffic": ncu_traffic(dc["case"], args.op) if args.path == "auto" else None,
-                "algorithmic_bytes": achieved}
+    traffic = ncu_traffic(dc["case"], args.op, detail=True) if args.path == "auto" else None
+    roofline = roofline_entry(kname, dc["case"], dc["read_bytes"] + dc["written_bytes"], avg[dom], peak, peak_src,
+                              traffic)
 
     if args.op == "inverse":
         for cl in calls:
@@ -457,9 +551,12 @@ def run_ours(args, rank, world, local):
                    "bytes_per_step": step_bytes, "bytes_per_step_pages_convention": step_bytes_pages,
                    "l2": "inputs/outputs rotate per call over " + ", ".join(str(len(r)) for r in rot)
                          + f" copies ({rot_bytes / 1e6:.0f} MB); each call's rotation alone spans > 4x L2",
-                   "timing": "one CUDA graph of all timed steps between two CUDA events, max over ranks; "
-                             "per-call durations from one graph per call type (same launches, back to back)"},
+                   "timing": "the timed steps: one CUDA graph (uploaded beforehand) replayed once between two CUDA "
+                             "events after the warm-up graph, max over ranks; per-call durations: each call's "
+                             f"launches back to back in a graph of their own ({n_call} launches, same rotation), "
+                             "one untimed replay, then one timed replay"},
         "frac_of_peak": round(value / world / peak, 4),
+        "frac_of_nominal": round(value / world / NOMINAL_HBM_GBS, 4),
         "calls": calls,
         "roofline": roofline,
         "e2e": e2e,
@@ -468,6 +565,135 @@ def run_ours(args, rank, world, local):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(cases, args.cpu_seconds)
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result))
+
+
+SWEEP_MAX_COPIES = 64            # rotation cap per sweep point (small points stay L2-warm)
+SWEEP_GRAPH_SECONDS = 0.02       # about this much work per timing graph
+SWEEP_ORACLE_SINGLE_RUN = 256e6  # traffic above which the oracle is timed on one run
+
+
+def sweep_launches(traffic_bytes: int) -> int:
+    """Launches per timing graph of a sweep point: about SWEEP_GRAPH_SECONDS of
+    work at an assumed 4 TB/s plus 3 us per launch, between 20 and 2000."""
+    est = 3e-6 + traffic_bytes / 4e12
+    return int(min(2000, max(20, SWEEP_GRAPH_SECONDS / est)))
+
+
+def oracle_seconds(case) -> tuple[float, str]:
+    """Single-thread CPU oracle time of one full call: the median of 3 runs
+    (each repeated to at least 20 ms for tiny points), or one run above
+    SWEEP_ORACLE_SINGLE_RUN bytes of traffic."""
+    import oracle
+
+    oracle.load()
+    b = algorithmic_bytes(case)
+    if b["read"] + b["written"] > SWEEP_ORACLE_SINGLE_RUN:
+        t0 = time.perf_counter()
+        oracle.rearrange(case.dim, case.scales, case.ends)
+        return time.perf_counter() - t0, "1 run"
+    t0 = time.perf_counter()
+    oracle.rearrange(case.dim, case.scales, case.ends)
+    once = max(time.perf_counter() - t0, 1e-7)
+    reps = max(1, int(math.ceil(0.02 / once)))
+    runs = []
+    for _ in range(3):
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            oracle.rearrange(case.dim, case.scales, case.ends)
+        runs.append((time.perf_counter() - t0) / reps)
+    return statistics.median(runs), f"median of 3 runs of {reps}"
+
+
+def run_sweep(args, rank, world, device, dist):
+    """Every point of the K-groups sweep, one after another: per point, its
+    launches back to back in one uploaded graph over a rotation of input and
+    output copies (one untimed replay, one timed), a same-size device copy
+    timed the same way, and the CPU oracle on the host."""
+    import torch
+
+    from scale_factor_layout_b200 import synth
+
+    peak, peak_src = load_peaks()
+    stream = torch.cuda.Stream(device)
+    h = stream.cuda_stream
+    timer = GraphTimer(stream, dist, device)
+    points, total_bytes, total_s, launches = [], 0, 0.0, 0
+    sampler = ClockSampler(device.index)
+    with sampler:
+        t_start = time.perf_counter()
+        for i_m, i_k in synth.sweep_points():
+            case = synth.k_sweep_point(i_m, i_k)
+            b = algorithmic_bytes(case)
+            traffic = b["read"] + b["written"]
+            per_copy = b["read"] + b["alloc"]
+            n_rot = min(max(2, math.ceil(4 * L2_BYTES / per_copy)), SWEEP_MAX_COPIES)
+            rot = device_copies(case, n_rot, device)
+            with torch.cuda.stream(stream):
+                launch(rot[0], h)
+            n = sweep_launches(traffic)
+            g = timer.capture([lambda it=rot[k % n_rot]: launch(it, h) for k in range(n)])
+            t = timer.steady(g, n)
+            del g
+            srcs = [it[1] for it in rot]
+            dsts = [torch.empty_like(x) for x in srcs]
+            g = timer.capture([lambda a=srcs[k % n_rot], d=dsts[k % n_rot]: d.copy_(a) for k in range(n)])
+            t_copy = timer.steady(g, n)
+            del g, dsts, srcs, rot
+            torch.cuda.empty_cache()
+            entry = {"M": case.extra["M"], "TotalK": case.extra["TotalK"], "rows": case.rows, "cols": case.cols,
+                     "us": round(t * 1e6, 3), "gbps": round(traffic / t / 1e9, 1),
+                     "frac_of_peak": round(traffic / t / 1e9 / peak, 4),
+                     "frac_of_nominal": round(traffic / t / 1e9 / NOMINAL_HBM_GBS, 4),
+                     "gbps_pages_convention": round(per_copy / t / 1e9, 1),
+                     "read_bytes": b["read"], "written_bytes": b["written"], "alloc_bytes": b["alloc"],
+                     "copy_us": round(t_copy * 1e6, 3),
+                     "frac_of_copy": round((2 * case.rows * case.cols / t_copy) / (traffic / t), 4),
+                     "launches_timed": n, "rotation": n_rot, "l2_cold": n_rot * per_copy >= 4 * L2_BYTES}
+            if rank == 0 and not args.no_cpu_baseline:
+                ts, how = oracle_seconds(case)
+                entry.update({"oracle_us": round(ts * 1e6, 1), "oracle_gbps": round(traffic / ts / 1e9, 3),
+                              "oracle_runs": how})
+            points.append(entry)
+            total_bytes += traffic
+            total_s += t
+            launches += n
+        sampler.window = (t_start, time.perf_counter())
+    big = [p for p in points if p["read_bytes"] + p["written_bytes"] >= 32e6]
+    result = {
+        "metric": METRIC, "value": round(total_bytes / total_s / 1e9, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": 1, "warmup": args.warmup, "ms_per_step": round(total_s * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+        "data": "synthetic (seeded uniform E8M0 bytes, seeded group splits)",
+        "config": {"workload": "k_sweep", "op": "rearrange", "path": "auto",
+                   "description": "K-groups sweep: M in {128..28672} x TotalK in {2^10..2^19}, scales M x TotalK/32, "
+                                  "G=8 (70 points); a step is one pass over every point",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "bytes_per_step": total_bytes,
+                   "l2": f"per point, inputs/outputs rotate over copies spanning >= 4x L2 where at most "
+                         f"{SWEEP_MAX_COPIES} copies suffice (l2_cold), else over {SWEEP_MAX_COPIES} copies",
+                   "timing": "per point: its launches back to back in one uploaded CUDA graph, one untimed replay, "
+                             "one timed replay between CUDA events; value = all points' bytes / the sum of their "
+                             "per-launch times"},
+        "frac_of_peak": round(total_bytes / total_s / 1e9 / peak, 4),
+        "points": points,
+        "large_points_min_frac_of_peak": min((p["frac_of_peak"] for p in big), default=None),
+        "roofline": roofline_entry("rearrange_tma_k", "k_sweep, all points", total_bytes, total_s, peak, peak_src,
+                                   None),
+        "e2e": None,
+        "gpu_launches": launches,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        t_cpu = sum(p["oracle_us"] for p in points) * 1e-6
+        result["cpu_baseline"] = {"value": round(total_bytes / t_cpu / 1e9, 3), "unit": "GB/s", "cores": 1,
+                                  "kind": "oracle",
+                                  "sample": f"every sweep point once (median of 3 below {SWEEP_ORACLE_SINGLE_RUN/1e6:.0f} "
+                                            f"MB of traffic), single thread, gcc -O2, {os.cpu_count()} host cores "
+                                            f"({cpu_model()})"}
     if dist is not None:
         dist.destroy_process_group()
     if rank == 0:
@@ -651,7 +877,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=workload_arg, default="moe_step",
-                    help=f"one of {sorted(WORKLOADS)} or k_sweep_<M>x<TotalK> (a point of the K-groups sweep)")
+                    help=f"one of {sorted(WORKLOADS)}, k_sweep (all 70 points of the K-groups sweep) "
+                         "or k_sweep_<M>x<TotalK> (one point)")
     ap.add_argument("--op", choices=["rearrange", "inverse"], default="rearrange",
                     help="rearrange (row-major -> blocked, the hot path) or its inverse")
     ap.add_argument("--path", choices=["auto", "tma", "flat", "word", "byte"], default="auto",
@@ -662,6 +889,8 @@ def main(argv=None):
     ap.add_argument("--no-copy-ceiling", action="store_true",
                     help="skip timing a same-size device-to-device copy per call")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--call-launches", type=int, default=2000,
+                    help="minimum launches in each per-call timing graph (steady-state per-launch duration)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     args.steps = max(1, args.steps)

@@ -48,7 +48,18 @@
  * Errors.  Argument faults the host can see return a status and launch
  * nothing.  A failed CUDA call returns MX_ERR_CUDA (mx_last_cuda_error gives
  * the CUDA code).
- * Bad device-side offsets are clamped as stated above.
+ * Bad device-side offsets are clamped as stated above.  Every wait of a
+ * kernel's copy pipeline has a time limit (about 2^31 SM clocks); a kernel
+ * whose wait runs out sets bit 0 of the device flags and returns early, and
+ * the output of that call is then undefined (partly written).  The call
+ * itself has already returned MX_OK by then: the flags (mx_device_flags) are
+ * the only record, and they are shared by every call on the device, so check
+ * them after a batch of calls, not per call.
+ *
+ * Contexts.  The library uses the CUDA context current in the calling
+ * thread.  Only when no context is current does it bind the current
+ * device's primary context (as the CUDA runtime would); a context the caller
+ * made current, primary or not, is left in place.
  */
 #ifndef MXSCALE_H
 #define MXSCALE_H
@@ -154,9 +165,11 @@ mx_path mx_select_path(mx_group_dim dim, const void *scales, int64_t rows, int64
 const char *mx_status_string(mx_status status);
 
 /* Device-side error flags of the current device (bit 0: a pipeline wait ran
- * past its time limit and the kernel returned early).  Synchronises the
- * device: for tests and debugging, never on a hot path.  `clear` != 0 resets
- * the flags after reading. */
+ * past its time limit and the kernel returned early; the output of the call
+ * that set it is undefined).  The flags accumulate over every call of every
+ * thread on the device until cleared, so a set bit names no call.
+ * Synchronises the device: for tests and debugging, never on a hot path.
+ * `clear` != 0 resets the flags after reading. */
 mx_status mx_device_flags(uint32_t *flags, int clear);
 
 /* Failure-detection self-test: launches one CTA that waits, with the same

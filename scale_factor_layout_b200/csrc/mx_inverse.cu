@@ -576,6 +576,257 @@ unrearrange_tma_m_kernel(const __grid_constant__ CUtensorMap omap, int64_t map_w
     unrearrange_body<true, 8, true>(&omap, map_w, blocked, blocked_size, ends, scales, row_stride, s, mode);
 }
 
+// ------------------------------------------------------------------ K-groups, output boxes
+// Groups along K into an output whose base is 16-byte aligned and whose row
+// stride is a multiple of 16 (the usual case): work items are boxes of the
+// OUTPUT, 128 rows x 128 columns, so that each is written with one 2-D tensor
+// store and no byte of the output has two writers.  The columns of a box
+// belong to one or more groups ("pieces"); a piece's tiles of the box's row
+// band are one contiguous span of the blocked buffer (group g's tiles
+// (rb, t) at R*Q_g + rb*128*W_g + 512*t), loaded with one bulk copy each into
+// the item's stage.  Per 16-byte output chunk of a row (16 consecutive
+// columns of one group's row), five consecutive tiles' words and a funnel
+// shift give the bytes, as in the shift-mode transpose above; a chunk that
+// holds a seam merges the pieces' bytes by column.  Columns no group covers
+// are zero.  A box with more pieces than kBoxPieces, or more tiles than a
+// stage holds (groups narrower than about 40 columns), is gathered byte by
+// byte from global memory instead.
+constexpr int kBoxPieces = 4;
+constexpr int kBoxStageTiles = 40;                    // 32 + 1.5 per piece, rounded up
+constexpr int kBoxStageBytes = kBoxStageTiles * 512;  // 20 KB
+constexpr int kBoxBlockBytes = kTileRows * 128;       // 16 KB, 128B-swizzled rows of 128 bytes
+constexpr int kBoxSmemBytes = kInvStages * kBoxStageBytes + 2 * kBoxBlockBytes + 1024;
+
+struct BoxPiece {
+    int32_t c0, c1;   // output columns [c0, c1) of the piece
+    int32_t g;        // its group
+    int32_t b;        // the group's first column
+    int32_t f;        // first tile of the group loaded (local tile index)
+    int32_t ntl;      // tiles loaded
+    int32_t s0;       // stage tile holding tile f
+};
+
+struct BoxItem {
+    int32_t x, y;     // first output column (a multiple of 128) and row
+    int32_t ncols;    // columns of the box inside the output (<= 128)
+    int32_t np;       // pieces, or -1: gather the box from global memory
+    int32_t rb;       // row band
+    int32_t tiles;    // tiles loaded into the stage
+    BoxPiece p[kBoxPieces];
+};
+
+// The group that holds column c, for 0 <= c < E'[G-1]: the last group whose
+// first column is <= c (begin[] is non-decreasing; that group is never an
+// empty one, whose successor starts at the same column).
+__device__ __forceinline__ int find_group_col(const GroupTable &t, int G, int c) {
+    int lo = 0, hi = G;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (t.begin[mid] <= c) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+// Work item i (row band i / nbox, column box i % nbox), written in place
+// (shared memory) by the one thread that decodes.
+__device__ __forceinline__ void decode_box(const GroupTable &t, const Shape &s, int nbox, int i, BoxItem &it) {
+    it.rb = i / nbox;
+    it.x = (i - it.rb * nbox) * 128;
+    it.y = it.rb * kTileRows;
+    it.ncols = min(128, s.cols - it.x);
+    it.np = 0;
+    it.tiles = 0;
+    const int used = t.begin[s.G - 1] + t.size[s.G - 1];
+    const int xend = it.x + it.ncols;
+    if (it.x >= used) return;
+    for (int g = find_group_col(t, s.G, it.x); g < s.G && t.begin[g] < xend; ++g) {
+        if (t.size[g] == 0) continue;
+        if (it.np == kBoxPieces) {
+            it.np = -1;
+            return;
+        }
+        BoxPiece &p = it.p[it.np];
+        p.g = g;
+        p.b = t.begin[g];
+        p.c0 = max(it.x, p.b);
+        p.c1 = min(xend, p.b + t.size[g]);
+        p.f = (p.c0 - p.b) >> 2;
+        p.ntl = ((p.c1 - 1 - p.b) >> 2) - p.f + 1;
+        p.s0 = it.tiles;
+        it.tiles += p.ntl;
+        if (it.tiles > kBoxStageTiles) {
+            it.np = -1;
+            return;
+        }
+        ++it.np;
+    }
+}
+
+// Byte offset in the blocked buffer of local tile `tl` of group g in row band rb.
+__device__ __forceinline__ int64_t box_src(const GroupTable &t, const Shape &s, int g, int rb, int tl) {
+    const int W = t.pstart[g + 1] - t.pstart[g];
+    return (int64_t)s.padded_rows * t.pstart[g] + (int64_t)rb * kTileRows * W + 512ll * tl;
+}
+
+__global__ void __launch_bounds__(kThreads, 3)
+unrearrange_box_k_kernel(const __grid_constant__ CUtensorMap omap, const uint8_t *__restrict__ blocked,
+                         const int32_t *__restrict__ ends, uint8_t *__restrict__ scales, int64_t row_stride,
+                         Shape s) {
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t *stages = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+    uint8_t *rowblks = stages + kInvStages * kBoxStageBytes;
+    __shared__ GroupTable table;
+    __shared__ __align__(8) uint64_t full[kInvStages];
+    __shared__ BoxItem items[kInvStages + 1];   // [kInvStages]: the next refill, decoded ahead
+    const int tid = threadIdx.x;
+    const int j = tid & 31;
+    const int q = tid >> 5;   // warp q makes output chunk q of every row
+
+    if (tid == 0) {
+        tma_prefetch_desc(&omap);
+#pragma unroll
+        for (int st = 0; st < kInvStages; ++st) mbar_init(&full[st], 1);
+        fence_mbar_init();
+    }
+    grid_dependency_wait();
+    if (q == 0) build_group_table<false>(ends, s.G, s.cols, 1, table);
+    __syncthreads();
+    grid_launch_dependents();
+    const int nbox = (s.cols + 127) >> 7;
+    const int total = (s.padded_rows / kTileRows) * nbox;
+    const int bid = blockIdx.x;
+    const int n_my = bid < total ? (total - 1 - bid) / (int)gridDim.x + 1 : 0;
+    const int partial_m = (s.cols & 15) ? ((s.cols & 127) >> 4) : -1;   // chunk of the last box cut by cols
+
+    // thread 0: stage st's item is items[st]; start its copies
+    auto issue = [&](int st) {
+        const BoxItem &it = items[st];
+        const uint32_t bytes = it.np > 0 ? (uint32_t)it.tiles * 512u : 0u;
+        mbar_arrive_expect_tx(&full[st], bytes);
+        for (int k = 0; k < it.np; ++k)
+            bulk_load_g2s(stages + st * kBoxStageBytes + it.p[k].s0 * 512,
+                          blocked + box_src(table, s, it.p[k].g, it.rb, it.p[k].f), (uint32_t)it.p[k].ntl * 512u,
+                          &full[st]);
+    };
+    if (tid == 0)
+        for (int st = 0; st < kInvStages && st < n_my; ++st) {
+            decode_box(table, s, nbox, bid + st * (int)gridDim.x, items[st]);
+            issue(st);
+        }
+
+    for (int n = 0; n < n_my; ++n) {
+        const int st = n % kInvStages;
+        const bool refill = tid == 0 && n + kInvStages < n_my;
+        if (refill) decode_box(table, s, nbox, bid + (n + kInvStages) * (int)gridDim.x, items[kInvStages]);
+        const bool ok = mbar_wait_bounded(&full[st], (uint32_t)(n / kInvStages) & 1u);
+        uint8_t *rowblk = rowblks + (n & 1) * kBoxBlockBytes;
+        // the item's scalars in registers: items[st] is refilled after the barrier
+        int ix = 0, iy = 0, incols = 0;
+        if (ok) {
+            const BoxItem &it = items[st];
+            ix = it.x;
+            iy = it.y;
+            incols = it.ncols;
+            const uint8_t *stage = stages + st * kBoxStageBytes;
+            const int cc0 = it.x + 16 * q;   // first column of this warp's chunk
+            uint4 o[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) o[a] = make_uint4(0u, 0u, 0u, 0u);
+            if (it.np > 0 && cc0 < it.x + it.ncols) {
+                for (int k = 0; k < it.np; ++k) {
+                    const BoxPiece &p = it.p[k];
+                    if (p.c1 <= cc0 || p.c0 >= cc0 + 16) continue;
+                    const int u = cc0 - p.b;           // local column of the chunk's byte 0 (may be < 0)
+                    const int t0 = u >> 2;             // floor
+                    const int sh = (u & 3) * 8;
+                    uint4 w[5];
+#pragma unroll
+                    for (int t = 0; t < 5; ++t) {
+                        const int tl = t0 + t - p.f;   // tile within the piece's loaded run
+                        w[t] = (tl >= 0 && tl < p.ntl && (t < 4 || sh != 0))
+                                   ? *reinterpret_cast<const uint4 *>(stage + (p.s0 + tl) * 512 + 16 * j)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    // bytes of the chunk that belong to this piece
+                    const int k0 = max(p.c0 - cc0, 0), k1 = min(p.c1 - cc0, 16);
+                    uint32_t keep[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int lo = min(max(k0 - 4 * e, 0), 4), hi = min(max(k1 - 4 * e, 0), 4);
+                        const uint32_t upto_hi = hi == 4 ? 0xffffffffu : (1u << (8 * hi)) - 1u;
+                        const uint32_t below_lo = lo == 4 ? 0xffffffffu : (1u << (8 * lo)) - 1u;
+                        keep[e] = upto_hi & ~below_lo;
+                    }
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        const uint32_t x0 = word_of(w[0], a), x1 = word_of(w[1], a), x2 = word_of(w[2], a),
+                                       x3 = word_of(w[3], a), x4 = word_of(w[4], a);
+                        o[a].x |= funnel(x0, x1, sh) & keep[0];
+                        o[a].y |= funnel(x1, x2, sh) & keep[1];
+                        o[a].z |= funnel(x2, x3, sh) & keep[2];
+                        o[a].w |= funnel(x3, x4, sh) & keep[3];
+                    }
+                }
+            } else if (it.np < 0 && cc0 < it.x + it.ncols) {
+                // many narrow groups: each byte straight from the blocked buffer
+                const int lim = min(table.begin[s.G - 1] + table.size[s.G - 1], it.x + it.ncols);
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    const int r = j + 32 * a;
+                    uint32_t wv[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const int c = cc0 + k;
+                        if (c < lim) {
+                            const int g = find_group_col(table, s.G, c);
+                            const int l = c - table.begin[g];
+                            const uint8_t v = __ldg(blocked + box_src(table, s, g, it.rb, l >> 2) + (r & 31) * 16 +
+                                                    (r >> 5) * 4 + (l & 3));
+                            wv[k >> 2] |= (uint32_t)v << (8 * (k & 3));
+                        }
+                    }
+                    o[a] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                }
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+                *reinterpret_cast<uint4 *>(rowblk + (j + 32 * a) * 128 + 16 * (q ^ (j & 7))) = o[a];
+            fence_proxy_async_smem();
+        }
+        // the tensor store of item n - 1 has read its row block, which item n + 1 overwrites
+        if (tid == 0) bulk_wait_read<0>();
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_inv_flags, kInvFlagWaitTimeout);
+                for (int m = n; m < n_my && m < n + kInvStages; ++m)
+                    mbar_wait_bounded(&full[m % kInvStages], (uint32_t)(m / kInvStages) & 1u);
+            }
+            return;
+        }
+        if (tid == 0) {
+            if (refill) {
+                items[st] = items[kInvStages];
+                issue(st);
+            }
+            // the map ends at the last whole 16-byte chunk of a row and at the last row
+            if (ix < (s.cols & ~15)) {
+                tma_store_2d(&omap, rowblk, ix, iy);
+                bulk_commit();
+            }
+        }
+        if (incols < 128 && partial_m >= 0 && tid < kTileRows) {
+            // the chunk that the output's last column cuts, past the map: byte stores
+            const int r = tid;
+            if (iy + r < s.rows) {
+                const uint8_t *src = rowblk + r * 128 + 16 * (partial_m ^ (r & 7));
+                uint8_t *dst = scales + (int64_t)(iy + r) * row_stride + ix + 16 * partial_m;
+                for (int k = 0; k < (s.cols & 15); ++k) dst[k] = src[k];
+            }
+        }
+    }
+    if (tid == 0) bulk_wait_all();
+}
+
 // One warp: the padded start of every group (rows for M, columns for K) and
 // the padded total, as int32[G + 1].
 template <bool kDimM>
@@ -612,9 +863,9 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // how many CTAs of them fit on an SM.
 constexpr int kMaxDevices = 128;
 std::mutex g_inv_mu;
-int g_inv_grid[kMaxDevices][3];   // SMs x resident CTAs: 8-warp, narrow, M tensor-store kernel; 0 until set up
+int g_inv_grid[kMaxDevices][4];   // SMs x resident CTAs: 8-warp, narrow, M tensor-store, K box kernel; 0 until set up
 
-enum InvKernel { kInvWide = 0, kInvNarrow = 1, kInvTmaM = 2 };
+enum InvKernel { kInvWide = 0, kInvNarrow = 1, kInvTmaM = 2, kInvBoxK = 3 };
 
 cudaError_t inverse_grid_cap(InvKernel which, int *cap) {
     int dev = 0;
@@ -622,7 +873,7 @@ cudaError_t inverse_grid_cap(InvKernel which, int *cap) {
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_inv_mu);
     if (g_inv_grid[dev][0] == 0) {
-        int sms = 0, occ_m = 0, occ_k = 0, occ_n = 0, occ_t = 0;
+        int sms = 0, occ_m = 0, occ_k = 0, occ_n = 0, occ_t = 0, occ_b = 0;
         const cudaError_t steps[] = {
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev),
             cudaFuncSetAttribute(unrearrange_kernel<true, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -633,18 +884,22 @@ cudaError_t inverse_grid_cap(InvKernel which, int *cap) {
                                  kInvNarrowSmemBytes),
             cudaFuncSetAttribute(unrearrange_tma_m_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kInvTmaSmemBytes),
+            cudaFuncSetAttribute(unrearrange_box_k_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kBoxSmemBytes),
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_m, unrearrange_kernel<true, 8>, kThreads, kInvSmemBytes),
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_k, unrearrange_kernel<false, 8>, kThreads, kInvSmemBytes),
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_n, unrearrange_kernel<true, 4>, 128, kInvNarrowSmemBytes),
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_t, unrearrange_tma_m_kernel, kThreads, kInvTmaSmemBytes),
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_b, unrearrange_box_k_kernel, kThreads, kBoxSmemBytes),
         };
         for (cudaError_t e : steps)
             if (e != cudaSuccess) return e;
         const int occ = occ_m < occ_k ? occ_m : occ_k;
-        if (occ < 1 || occ_n < 1 || occ_t < 1 || sms < 1) return cudaErrorInvalidConfiguration;
+        if (occ < 1 || occ_n < 1 || occ_t < 1 || occ_b < 1 || sms < 1) return cudaErrorInvalidConfiguration;
         g_inv_grid[dev][kInvWide] = sms * occ;
         g_inv_grid[dev][kInvNarrow] = sms * occ_n;
         g_inv_grid[dev][kInvTmaM] = sms * occ_t;
+        g_inv_grid[dev][kInvBoxK] = sms * occ_b;
     }
     *cap = g_inv_grid[dev][which];
     return cudaSuccess;
@@ -683,13 +938,33 @@ mx_status unrearrange(mx_group_dim dim, const uint8_t *blocked, int64_t rows, in
                                                                                                 : kModeRows;
     const bool narrow = mode == kModeFlat && s.padded_cols <= kInvNarrowCols;
     const bool tma_m = mode == kModeShift && dim_m;
+    // groups along K into a 16-byte aligned output: boxes of the output, one
+    // tensor store each (a map over the whole 16-byte chunks of each row)
+    const bool box_k = !dim_m && mode == kModeShift && (reinterpret_cast<uintptr_t>(scales) & 15u) == 0 &&
+                       cols >= 16 && row_stride < (1ll << 40);
     int cap = 0;
-    if (cudaError_t e = inverse_grid_cap(narrow ? kInvNarrow : tma_m ? kInvTmaM : kInvWide, &cap); e != cudaSuccess)
+    if (cudaError_t e = inverse_grid_cap(box_k    ? kInvBoxK
+                                         : narrow ? kInvNarrow
+                                         : tma_m  ? kInvTmaM
+                                                  : kInvWide,
+                                         &cap);
+        e != cudaSuccess)
         return mx_record_cuda_error(e);
-    const int grid = (int)(bound < 1 ? 1 : (bound < cap ? bound : cap));
+    const int64_t box_bound = ceil_div(rows, 128) * ceil_div(cols, 128);
+    const int64_t work = box_k ? box_bound : bound;
+    const int grid = (int)(work < 1 ? 1 : (work < cap ? work : cap));
     const int64_t blocked_size = (int64_t)mx_rearranged_size(dim, rows, cols, G);
     cudaError_t e;
-    if (tma_m) {
+    if (box_k) {
+        CUtensorMap omap;
+        std::memset(&omap, 0, sizeof(omap));
+        if (mx_status st = mx_encode_rows_map(&omap, scales, cols & ~int64_t(15), rows, row_stride, 128, 128,
+                                              CU_TENSOR_MAP_SWIZZLE_128B);
+            st != MX_OK)
+            return st;
+        e = launch_kernel(unrearrange_box_k_kernel, grid, kThreads, kBoxSmemBytes, stream, omap, blocked, ends, scales,
+                          row_stride, s);
+    } else if (tma_m) {
         // Whole-box items go out as tensor stores: a map over the output from
         // the 16-byte boundary at or below its first byte, as wide as the rows
         // reach (capped at the row stride; items past the cap use plain stores).

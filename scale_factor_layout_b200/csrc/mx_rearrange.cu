@@ -689,17 +689,34 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return g_encode;
 }
 
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+std::once_flag g_ctx_once;
+
+PFN_cuCtxGetCurrent_v4000 ctx_current_fn() {
+    std::call_once(g_ctx_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    });
+    return g_ctx_current;
+}
+
 mx_status device_info(const DeviceInfo **out) {
     int dev = 0;
     if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
     if (dev < 0 || dev >= kMaxDevices) return MX_ERR_UNSUPPORTED;
-    // The tensor-map encoder is a driver call and needs the device's primary
-    // context current in this thread; a thread whose first CUDA work is this
-    // call has none yet, so bind it once per thread and device.
-    thread_local int t_bound_dev = -1;
-    if (t_bound_dev != dev) {
+    // The tensor-map encoder is a driver call and needs a context current in
+    // this thread.  A thread whose first CUDA work is this call has none yet:
+    // bind the device's primary context then, and only then, so that a
+    // context the caller made current (the primary one or its own) stays.
+    auto get_current = ctx_current_fn();
+    if (get_current == nullptr) return cuda_status(cudaErrorSymbolNotFound);
+    CUcontext cur = nullptr;
+    if (CUresult r = get_current(&cur); r != CUDA_SUCCESS) return cuda_status(static_cast<cudaError_t>(r));
+    if (cur == nullptr) {
         if (cudaError_t e = cudaSetDevice(dev); e != cudaSuccess) return cuda_status(e);
-        t_bound_dev = dev;
     }
     std::lock_guard<std::mutex> lock(g_mu);
     DeviceInfo &d = g_dev[dev];

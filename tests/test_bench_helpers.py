@@ -73,3 +73,39 @@ def test_algorithmic_bytes_match_the_oracle(orc):
         assert b["read"] == orc.read_bytes(c.dim, c.rows, c.cols, c.ends), c.name
         assert b["written"] == orc.written_bytes(c.dim, c.rows, c.cols, c.ends), c.name
         assert b["alloc"] == orc.rearranged_size(c.dim, c.rows, c.cols, len(c.ends)), c.name
+
+
+def test_traffic_detail_and_roofline_fields(tmp_path):
+    """The roofline object carries read and write traffic apart, flags a
+    launch whose writes are still in L2 when it ends, and gives the fraction
+    of the nominal peak beside the measured one."""
+    _copy_tree(tmp_path)
+    fwd, _ = _keys(str(tmp_path))
+    traffic = tmp_path / "traffic.txt"
+    traffic.write_text(f"op=rearrange call=k_groups bytes_per_launch=1068 read=1000 write=68 l2_write=998 "
+                       f"source_sha={fwd} capture=a.md\n"
+                       f"op=rearrange call=m_wide bytes_per_launch=2000 read=1000 write=1000 "
+                       f"source_sha={fwd} capture=b.md\n")
+    root, path = str(tmp_path), str(traffic)
+    t = bench.ncu_traffic("k_groups", "rearrange", root, path, detail=True)
+    assert t == {"read": 1000, "write": 68, "l2_write": 998}
+    assert bench.ncu_traffic("m_wide", "rearrange", root, path, detail=True)["l2_write"] is None
+    r = bench.roofline_entry("k", "k_groups", 2000, 1e-6, 4000.0, "measured", t)
+    assert r["achieved"] == 2.0 and r["frac"] == round(2.0 / 4000.0, 4)
+    assert r["frac_of_nominal"] == round(2.0 / bench.NOMINAL_HBM_GBS, 4)
+    assert (r["traffic"], r["traffic_read"], r["traffic_write"], r["traffic_l2_write"]) == (1068, 1000, 68, 998)
+    assert "traffic_note" in r
+    full = bench.roofline_entry("k", "m_wide", 2000, 1e-6, 4000.0, "measured",
+                                bench.ncu_traffic("m_wide", "rearrange", root, path, detail=True))
+    assert "traffic_note" not in full and "traffic_l2_write" not in full
+    assert bench.roofline_entry("k", "x", 2000, 1e-6, 4000.0, "measured", None)["traffic"] is None
+
+
+def test_timing_graph_sizes():
+    """Per-call timing graphs hold at least the minimum launch count; sweep
+    graphs hold about 20 ms of work, between 20 and 2000 launches."""
+    assert bench.per_launch_launches(20, 2000) == 2000
+    assert bench.per_launch_launches(4000, 2000) == 4000
+    assert bench.sweep_launches(8192) == 2000
+    assert bench.sweep_launches(940_000_000) == 84
+    assert bench.sweep_launches(10**12) == 20

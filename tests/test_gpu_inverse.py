@@ -85,6 +85,29 @@ def test_inverse_narrow_k_groups(mxlib, orc, misalign):
     _inverse_check(case, orc, out_pad=(-cols) % 16 + 16, misalign=misalign)
 
 
+@pytest.mark.parametrize("seed", range(12))
+def test_inverse_k_output_boxes(mxlib, orc, seed):
+    """Groups along K into a 16-byte aligned output with a row stride that is a
+    multiple of 16: the kernel that writes 128 x 128 boxes of the output with
+    tensor stores.  Widths from 16 to 1100 columns (a last chunk cut by the
+    width, boxes narrower than 128), groups from one column wide to wider than
+    a box (so boxes hold one to many pieces, beyond what a stage takes), empty
+    groups, columns no group covers, and rows that end inside a row band."""
+    rng = np.random.default_rng(4600 + seed)
+    rows = int(rng.integers(1, 700))
+    cols = int(rng.choice([16, 17, 40, 127, 128, 129, 300, 512, 1100, int(rng.integers(16, 1200))]))
+    G = int(rng.integers(1, 65))
+    narrow = seed % 3 == 0
+    widths = rng.integers(0, 12 if narrow else 2 * cols // G + 2, size=G)
+    widths[rng.random(G) < 0.15] = 0
+    while widths.sum() > cols:
+        widths[int(rng.integers(0, G))] //= 2
+    scales = rng.integers(1, 255, size=(rows, cols), dtype=np.uint8)
+    case = synth.Case("boxK", synth.DIM_K, scales, np.cumsum(widths).astype(np.int32), 0)
+    for pad in ((-cols) % 16, (-cols) % 16 + 16):
+        _inverse_check(case, orc, out_pad=pad, misalign=0)
+
+
 def test_inverse_ignores_padding_values(mxlib, orc):
     """Padding bytes of the blocked buffer (and its tail) filled with garbage
     change nothing: the inverse reads whole tiles but writes only real data."""
