@@ -598,8 +598,8 @@ constexpr int kBoxBlockBytes = kTileRows * 128;       // 16 KB, 128B-swizzled ro
 constexpr int kBoxSmemBytes = kInvStages * kBoxStageBytes + 2 * kBoxBlockBytes + 1024;
 
 struct BoxPiece {
+    int64_t src;      // blocked offset of the first tile loaded
     int32_t c0, c1;   // output columns [c0, c1) of the piece
-    int32_t g;        // its group
     int32_t b;        // the group's first column
     int32_t f;        // first tile of the group loaded (local tile index)
     int32_t ntl;      // tiles loaded
@@ -627,6 +627,12 @@ __device__ __forceinline__ int find_group_col(const GroupTable &t, int G, int c)
     return lo;
 }
 
+// Byte offset in the blocked buffer of local tile `tl` of group g in row band rb.
+__device__ __forceinline__ int64_t box_src(const GroupTable &t, const Shape &s, int g, int rb, int tl) {
+    const int W = t.pstart[g + 1] - t.pstart[g];
+    return (int64_t)s.padded_rows * t.pstart[g] + (int64_t)rb * kTileRows * W + 512ll * tl;
+}
+
 // Work item i (row band i / nbox, column box i % nbox), written in place
 // (shared memory) by the one thread that decodes.
 __device__ __forceinline__ void decode_box(const GroupTable &t, const Shape &s, int nbox, int i, BoxItem &it) {
@@ -646,11 +652,11 @@ __device__ __forceinline__ void decode_box(const GroupTable &t, const Shape &s, 
             return;
         }
         BoxPiece &p = it.p[it.np];
-        p.g = g;
         p.b = t.begin[g];
         p.c0 = max(it.x, p.b);
         p.c1 = min(xend, p.b + t.size[g]);
         p.f = (p.c0 - p.b) >> 2;
+        p.src = box_src(t, s, g, it.rb, p.f);
         p.ntl = ((p.c1 - 1 - p.b) >> 2) - p.f + 1;
         p.s0 = it.tiles;
         it.tiles += p.ntl;
@@ -662,12 +668,6 @@ __device__ __forceinline__ void decode_box(const GroupTable &t, const Shape &s, 
     }
 }
 
-// Byte offset in the blocked buffer of local tile `tl` of group g in row band rb.
-__device__ __forceinline__ int64_t box_src(const GroupTable &t, const Shape &s, int g, int rb, int tl) {
-    const int W = t.pstart[g + 1] - t.pstart[g];
-    return (int64_t)s.padded_rows * t.pstart[g] + (int64_t)rb * kTileRows * W + 512ll * tl;
-}
-
 __global__ void __launch_bounds__(kThreads, 3)
 unrearrange_box_k_kernel(const __grid_constant__ CUtensorMap omap, const uint8_t *__restrict__ blocked,
                          const int32_t *__restrict__ ends, uint8_t *__restrict__ scales, int64_t row_stride,
@@ -677,10 +677,11 @@ unrearrange_box_k_kernel(const __grid_constant__ CUtensorMap omap, const uint8_t
     uint8_t *rowblks = stages + kInvStages * kBoxStageBytes;
     __shared__ GroupTable table;
     __shared__ __align__(8) uint64_t full[kInvStages];
-    __shared__ BoxItem items[kInvStages + 1];   // [kInvStages]: the next refill, decoded ahead
+    __shared__ BoxItem items[kInvStages + 1];   // item n in slot n % 3
     const int tid = threadIdx.x;
     const int j = tid & 31;
     const int q = tid >> 5;   // warp q makes output chunk q of every row
+    constexpr int kSlots = kInvStages + 1;
 
     if (tid == 0) {
         tma_prefetch_desc(&omap);
@@ -698,32 +699,36 @@ unrearrange_box_k_kernel(const __grid_constant__ CUtensorMap omap, const uint8_t
     const int n_my = bid < total ? (total - 1 - bid) / (int)gridDim.x + 1 : 0;
     const int partial_m = (s.cols & 15) ? ((s.cols & 127) >> 4) : -1;   // chunk of the last box cut by cols
 
-    // thread 0: stage st's item is items[st]; start its copies
-    auto issue = [&](int st) {
-        const BoxItem &it = items[st];
+    // thread 0: start the copies of item n (slot n % 3) into stage n % 2
+    auto issue = [&](int n) {
+        const BoxItem &it = items[n % kSlots];
+        const int st = n % kInvStages;
         const uint32_t bytes = it.np > 0 ? (uint32_t)it.tiles * 512u : 0u;
         mbar_arrive_expect_tx(&full[st], bytes);
         for (int k = 0; k < it.np; ++k)
-            bulk_load_g2s(stages + st * kBoxStageBytes + it.p[k].s0 * 512,
-                          blocked + box_src(table, s, it.p[k].g, it.rb, it.p[k].f), (uint32_t)it.p[k].ntl * 512u,
-                          &full[st]);
+            bulk_load_g2s(stages + st * kBoxStageBytes + it.p[k].s0 * 512, blocked + it.p[k].src,
+                          (uint32_t)it.p[k].ntl * 512u, &full[st]);
     };
     if (tid == 0)
-        for (int st = 0; st < kInvStages && st < n_my; ++st) {
-            decode_box(table, s, nbox, bid + st * (int)gridDim.x, items[st]);
-            issue(st);
+        for (int n = 0; n < kInvStages && n < n_my; ++n) {
+            decode_box(table, s, nbox, bid + n * (int)gridDim.x, items[n]);
+            issue(n);
         }
 
     for (int n = 0; n < n_my; ++n) {
         const int st = n % kInvStages;
-        const bool refill = tid == 0 && n + kInvStages < n_my;
-        if (refill) decode_box(table, s, nbox, bid + (n + kInvStages) * (int)gridDim.x, items[kInvStages]);
+        const bool refill = n + kInvStages < n_my;
+        // A thread of another warp than thread 0's decodes the refill into the
+        // slot that item n - 1 left, so that thread 0's work between two
+        // barriers is only the copies it issues.
+        if (refill && tid == 32)
+            decode_box(table, s, nbox, bid + (n + kInvStages) * (int)gridDim.x, items[(n + kInvStages) % kSlots]);
         const bool ok = mbar_wait_bounded(&full[st], (uint32_t)(n / kInvStages) & 1u);
         uint8_t *rowblk = rowblks + (n & 1) * kBoxBlockBytes;
         // the item's scalars in registers: items[st] is refilled after the barrier
         int ix = 0, iy = 0, incols = 0;
         if (ok) {
-            const BoxItem &it = items[st];
+            const BoxItem &it = items[n % kSlots];
             ix = it.x;
             iy = it.y;
             incols = it.ncols;
@@ -804,10 +809,7 @@ unrearrange_box_k_kernel(const __grid_constant__ CUtensorMap omap, const uint8_t
             return;
         }
         if (tid == 0) {
-            if (refill) {
-                items[st] = items[kInvStages];
-                issue(st);
-            }
+            if (refill) issue(n + kInvStages);
             // the map ends at the last whole 16-byte chunk of a row and at the last row
             if (ix < (s.cols & ~15)) {
                 tma_store_2d(&omap, rowblk, ix, iy);
