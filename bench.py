@@ -46,11 +46,13 @@ import numpy as np  # noqa: E402
 
 WORKLOADS = {
     "moe_step": ["m_skinny", "m_wide", "k_groups"],
+    "m_tiny": ["m_tiny"],
     "m_skinny": ["m_skinny"],
     "m_wide": ["m_wide"],
     "k_groups": ["k_groups"],
 }
 WORKLOAD_DESC = {
+    "m_tiny": "M-groups 1000x44 G=4 with one empty group, stride 44 B (flat-row TMA)",
     "moe_step": "M-groups 131072x44 G=8 (flat-row TMA) + M-groups 131072x224 G=8 (TMA) + K-groups 7168x4096 G=8 (TMA)",
     "m_skinny": "M-groups 131072x44 G=8, stride 44 B (flat-row TMA)",
     "m_wide": "M-groups 131072x224 G=8 (TMA)",
@@ -651,7 +653,7 @@ def run_sweep(args, rank, world, device, dist):
                      "gbps_pages_convention": round(per_copy / t / 1e9, 1),
                      "read_bytes": b["read"], "written_bytes": b["written"], "alloc_bytes": b["alloc"],
                      "copy_us": round(t_copy * 1e6, 3),
-                     "frac_of_copy": round((2 * case.rows * case.cols / t_copy) / (traffic / t), 4),
+                     "frac_of_copy": round((traffic / t) / (2 * case.rows * case.cols / t_copy), 4),
                      "launches_timed": n, "rotation": n_rot, "l2_cold": n_rot * per_copy >= 4 * L2_BYTES}
             if rank == 0 and not args.no_cpu_baseline:
                 ts, how = oracle_seconds(case)
