@@ -430,6 +430,16 @@ def roofline_entry(kernel: str, case_name: str, bytes_moved: int, seconds: float
     return out
 
 
+def inverse_kernel_name(case) -> str:
+    """The inverse kernel the library picks for a case written to a dense,
+    16-byte aligned row-major tensor (as the bench allocates it)."""
+    if case.dim == 1:
+        return "unrearrange_box_k_kernel" if case.cols >= 16 else "unrearrange_kernel<K, 8>"
+    if case.cols <= 128 and case.cols % 4 == 0:
+        return "unrearrange_kernel<M, 4>" if ceil_to(case.cols, 4) <= 48 else "unrearrange_kernel<M, 8>"
+    return "unrearrange_tma_m_kernel" if case.cols % 16 == 0 else "unrearrange_kernel<M, 8>"
+
+
 def run_ours(args, rank, world, local):
     import torch
 
@@ -532,7 +542,7 @@ def run_ours(args, rank, world, local):
     dc = calls[dom]
     kernel_names = {"tma": "rearrange_tma_m" if cases[dom].dim == 0 else "rearrange_tma_k",
                     "flat": "rearrange_flat_tma", "word": "rearrange_fallback", "byte": "rearrange_fallback"}
-    kname = "unrearrange_kernel" if args.op == "inverse" else kernel_names.get(dc["path"], "?")
+    kname = inverse_kernel_name(cases[dom]) if args.op == "inverse" else kernel_names.get(dc["path"], "?")
     traffic = ncu_traffic(dc["case"], args.op, detail=True) if args.path == "auto" else None
     roofline = roofline_entry(kname, dc["case"], dc["read_bytes"] + dc["written_bytes"], avg[dom], peak, peak_src,
                               traffic)
