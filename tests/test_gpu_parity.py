@@ -67,6 +67,24 @@ def test_k_sweep(mxlib, orc, i_rows):
         _check(synth.k_sweep_point(i_rows, i_k), orc)
 
 
+def test_k_groups_large_ragged(mxlib, orc):
+    """A 193 MiB K-groups input, whole output compared: rows that end inside
+    a row band, 64 groups from a few columns (quads that straddle group
+    boundaries) to hundreds wide, empty groups, columns that no group covers,
+    and gap bytes between rows."""
+    rng = np.random.default_rng(4700)
+    rows, cols, G = 16461, 12293, 64
+    widths = np.where(rng.random(G) < 0.5, rng.integers(0, 10, size=G), rng.integers(50, 600, size=G))
+    widths[rng.random(G) < 0.1] = 0
+    while widths.sum() > cols - 37:
+        widths[int(rng.integers(0, G))] //= 2
+    base = synth.Case("k_large", synth.DIM_K, np.zeros((rows, cols), np.uint8),
+                      np.cumsum(widths).astype(np.int32), 4700)
+    case = synth.strided(base, (-cols) % 16 + 16)
+    assert case.rows * case.cols >= 192 << 20 and case.row_stride % 16 == 0
+    _check(case, orc)
+
+
 @pytest.mark.parametrize("name,pad,path", [
     ("m_wide", 32, "auto"), ("k_groups", 32, "auto"),   # stride still a multiple of 16: TMA with gaps
     ("m_wide", 4, "auto"), ("k_groups", 4, "auto"),     # word path
