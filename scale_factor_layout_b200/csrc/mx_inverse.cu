@@ -590,7 +590,11 @@ unrearrange_tma_m_kernel(const __grid_constant__ CUtensorMap omap, int64_t map_w
 // holds a seam merges the pieces' bytes by column.  Columns no group covers
 // are zero.  A box with more pieces than kBoxPieces, or more tiles than a
 // stage holds (groups narrower than about 40 columns), is gathered byte by
-// byte from global memory instead.
+// byte from global memory instead.  Items go in group-major order (the boxes
+// whose first column lies in group 0, band after band, then group 1's, ...),
+// so that the items in flight read one stretch of the blocked buffer, which
+// lets each CTA prefetch its likely first tiles into L2 before its group
+// scan.
 constexpr int kBoxPieces = 4;
 constexpr int kBoxStageTiles = 40;                    // 32 + 1.5 per piece, rounded up
 constexpr int kBoxStageBytes = kBoxStageTiles * 512;  // 20 KB
@@ -635,9 +639,9 @@ __device__ __forceinline__ int64_t box_src(const GroupTable &t, const Shape &s, 
 
 // Work item i (row band i / nbox, column box i % nbox), written in place
 // (shared memory) by the one thread that decodes.
-__device__ __forceinline__ void decode_box(const GroupTable &t, const Shape &s, int nbox, int i, BoxItem &it) {
-    it.rb = i / nbox;
-    it.x = (i - it.rb * nbox) * 128;
+__device__ __forceinline__ void decode_box_at(const GroupTable &t, const Shape &s, int rb, int xb, BoxItem &it) {
+    it.rb = rb;
+    it.x = xb * 128;
     it.y = it.rb * kTileRows;
     it.ncols = min(128, s.cols - it.x);
     it.np = 0;
@@ -668,14 +672,57 @@ __device__ __forceinline__ void decode_box(const GroupTable &t, const Shape &s, 
     }
 }
 
+// Boxes per row band whose first column lies in group g (ceil(end/128) -
+// ceil(begin/128) for a non-empty group), and after the groups a last entry
+// for the boxes at or past the last clamped end; bs[g] is the exclusive
+// prefix, bs[G + 1] = boxes per band.  Warp 0, lanes holding g and g + 32.
+__device__ __forceinline__ void build_box_starts(const GroupTable &t, int G, int nbox, int32_t *bs) {
+    const int lane = threadIdx.x & 31;
+    auto nb = [&](int g) {
+        if (g >= G || t.size[g] == 0) return 0;
+        return (t.begin[g] + t.size[g] + 127) / 128 - (t.begin[g] + 127) / 128;
+    };
+    const int n0 = nb(lane), n1 = nb(lane + 32);
+    const int i0 = warp_scan_sum(n0, lane);
+    const int top = __shfl_sync(0xffffffffu, i0, 31);
+    const int i1 = warp_scan_sum(n1, lane) + top;
+    if (lane < G) bs[lane] = i0 - n0;
+    if (lane + 32 < G) bs[lane + 32] = i1 - n1;
+    if (lane == 31) {
+        const int used = t.begin[G - 1] + t.size[G - 1];
+        bs[G] = (used + 127) / 128;     // == i1 (boxes that start inside some group)
+        bs[G + 1] = nbox;
+    }
+}
+
+// Work item i in group-major order: the boxes of group 0 (whose first column
+// lies in it) band after band, then group 1's, ..., then the boxes past the
+// last group.  Items in flight then read one stretch of the blocked buffer.
+__device__ __forceinline__ void decode_box(const GroupTable &t, const Shape &s, const int32_t *bs, int bands, int i,
+                                           BoxItem &it) {
+    const int G = s.G;
+    int lo = 0, hi = G + 1;                       // last g in [0, G] with bands * bs[g] <= i
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (bands * bs[mid] <= i) lo = mid; else hi = mid;
+    }
+    while (lo < G && bs[lo + 1] == bs[lo]) ++lo;  // skip groups without boxes
+    const int nb = bs[lo + 1] - bs[lo];
+    const int local = i - bands * bs[lo];
+    const int rb = local / nb;
+    const int first = lo < G ? (t.begin[lo] + 127) / 128 : bs[G];
+    decode_box_at(t, s, rb, first + (local - rb * nb), it);
+}
+
 __global__ void __launch_bounds__(kThreads, 3)
 unrearrange_box_k_kernel(const __grid_constant__ CUtensorMap omap, const uint8_t *__restrict__ blocked,
-                         const int32_t *__restrict__ ends, uint8_t *__restrict__ scales, int64_t row_stride,
-                         Shape s) {
+                         int64_t blocked_size, const int32_t *__restrict__ ends, uint8_t *__restrict__ scales,
+                         int64_t row_stride, Shape s) {
     extern __shared__ uint8_t dyn_smem[];
     uint8_t *stages = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
     uint8_t *rowblks = stages + kInvStages * kBoxStageBytes;
     __shared__ GroupTable table;
+    __shared__ int32_t bstart[kMaxGroups + 2];
     __shared__ __align__(8) uint64_t full[kInvStages];
     __shared__ BoxItem items[kInvStages + 1];   // item n in slot n % 3
     const int tid = threadIdx.x;
@@ -689,11 +736,25 @@ unrearrange_box_k_kernel(const __grid_constant__ CUtensorMap omap, const uint8_t
         for (int st = 0; st < kInvStages; ++st) mbar_init(&full[st], 1);
         fence_mbar_init();
     }
+    // L2 prefetch of the blocked bytes this CTA most likely reads first: in
+    // group-major order item i's tiles lie near 16 KB * i (no observable
+    // value, so before the dependency wait)
+    if (tid == 32) {
+        for (int n = 0; n < kInvStages; ++n) {
+            const int64_t off = (int64_t)kBoxBlockBytes * ((int)blockIdx.x + n * (int)gridDim.x);
+            if (off + kBoxBlockBytes <= blocked_size) bulk_prefetch_l2(blocked + off, kBoxBlockBytes);
+        }
+    }
     grid_dependency_wait();
-    if (q == 0) build_group_table<false>(ends, s.G, s.cols, 1, table);
+    const int nbox = (s.cols + 127) >> 7;
+    if (q == 0) {
+        build_group_table<false>(ends, s.G, s.cols, 1, table);
+        __syncwarp();
+        build_box_starts(table, s.G, nbox, bstart);
+    }
     __syncthreads();
     grid_launch_dependents();
-    const int nbox = (s.cols + 127) >> 7;
+    const int bands = s.padded_rows / kTileRows;
     const int total = (s.padded_rows / kTileRows) * nbox;
     const int bid = blockIdx.x;
     const int n_my = bid < total ? (total - 1 - bid) / (int)gridDim.x + 1 : 0;
@@ -711,7 +772,7 @@ unrearrange_box_k_kernel(const __grid_constant__ CUtensorMap omap, const uint8_t
     };
     if (tid == 0)
         for (int n = 0; n < kInvStages && n < n_my; ++n) {
-            decode_box(table, s, nbox, bid + n * (int)gridDim.x, items[n]);
+            decode_box(table, s, bstart, bands, bid + n * (int)gridDim.x, items[n]);
             issue(n);
         }
 
@@ -722,7 +783,7 @@ unrearrange_box_k_kernel(const __grid_constant__ CUtensorMap omap, const uint8_t
         // slot that item n - 1 left, so that thread 0's work between two
         // barriers is only the copies it issues.
         if (refill && tid == 32)
-            decode_box(table, s, nbox, bid + (n + kInvStages) * (int)gridDim.x, items[(n + kInvStages) % kSlots]);
+            decode_box(table, s, bstart, bands, bid + (n + kInvStages) * (int)gridDim.x, items[(n + kInvStages) % kSlots]);
         const bool ok = mbar_wait_bounded(&full[st], (uint32_t)(n / kInvStages) & 1u);
         uint8_t *rowblk = rowblks + (n & 1) * kBoxBlockBytes;
         // the item's scalars in registers: items[st] is refilled after the barrier
@@ -964,8 +1025,8 @@ mx_status unrearrange(mx_group_dim dim, const uint8_t *blocked, int64_t rows, in
                                               CU_TENSOR_MAP_SWIZZLE_128B);
             st != MX_OK)
             return st;
-        e = launch_kernel(unrearrange_box_k_kernel, grid, kThreads, kBoxSmemBytes, stream, omap, blocked, ends, scales,
-                          row_stride, s);
+        e = launch_kernel(unrearrange_box_k_kernel, grid, kThreads, kBoxSmemBytes, stream, omap, blocked,
+                          blocked_size, ends, scales, row_stride, s);
     } else if (tma_m) {
         // Whole-box items go out as tensor stores: a map over the output from
         // the 16-byte boundary at or below its first byte, as wide as the rows
