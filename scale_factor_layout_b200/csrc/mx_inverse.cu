@@ -8,7 +8,9 @@
 // 512-byte lines (one warp reads one tile per 128-bit load), transposes 4x4
 // words in registers into a shared row block, and writes the output in
 // 16-byte aligned chunks that each have exactly one owning item (partial ones
-// as byte-masked bulk copies); the padded starts come from the same
+// as byte-masked bulk copies).  Groups along K into an aligned output take
+// another kernel, whose work items are 128x128 boxes of the output written
+// with one tensor store each.  The padded starts come from the same
 // warp-shuffle scan.
 
 #include <cuda.h>
@@ -637,8 +639,8 @@ __device__ __forceinline__ int64_t box_src(const GroupTable &t, const Shape &s, 
     return (int64_t)s.padded_rows * t.pstart[g] + (int64_t)rb * kTileRows * W + 512ll * tl;
 }
 
-// Work item i (row band i / nbox, column box i % nbox), written in place
-// (shared memory) by the one thread that decodes.
+// The box of row band rb and columns [128 xb, 128 xb + 128): its pieces,
+// written in place (shared memory) by the one thread that decodes.
 __device__ __forceinline__ void decode_box_at(const GroupTable &t, const Shape &s, int rb, int xb, BoxItem &it) {
     it.rb = rb;
     it.x = xb * 128;
@@ -724,7 +726,7 @@ unrearrange_box_k_kernel(const __grid_constant__ CUtensorMap omap, const uint8_t
     __shared__ GroupTable table;
     __shared__ int32_t bstart[kMaxGroups + 2];
     __shared__ __align__(8) uint64_t full[kInvStages];
-    __shared__ BoxItem items[kInvStages + 1];   // item n in slot n % 3
+    __shared__ BoxItem items[kInvStages + 1];   // item n in slot n % (kInvStages + 1)
     const int tid = threadIdx.x;
     const int j = tid & 31;
     const int q = tid >> 5;   // warp q makes output chunk q of every row
