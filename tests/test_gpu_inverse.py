@@ -170,3 +170,49 @@ def test_padded_group_starts(mxlib, orc):
         got = mxs.padded_group_starts(dim, rows, cols, torch.from_numpy(ends).cuda()).cpu().numpy()
         want = orc.padded_group_starts(dim, rows, cols, ends)
         assert np.array_equal(got.astype(np.int64), want), (dim, rows, cols, ends)
+
+
+def test_inverse_graph_capture(mxlib, orc):
+    """The inverse calls (output boxes along K, tensor-store boxes along M)
+    captured in one CUDA graph and replayed; group ends rewritten in place
+    between replays are read on the device by the next replay."""
+    rng = np.random.default_rng(4800)
+    cases = [synth.k_groups(), synth.m_wide()]
+    blocked, ends_d, outs = [], [], []
+    for c in cases:
+        e = torch.from_numpy(np.ascontiguousarray(c.ends, dtype=np.int32)).cuda()
+        blocked.append(torch.from_numpy(orc.rearrange(c.dim, c.scales, c.ends)).cuda())
+        ends_d.append(e)
+        outs.append(torch.empty((c.rows, c.cols), dtype=torch.uint8, device="cuda"))
+
+    def call(i, stream):
+        c = cases[i]
+        fn = B.mx_unrearrange_m_groups if c.dim == synth.DIM_M else B.mx_unrearrange_k_groups
+        st = fn(blocked[i].data_ptr(), c.rows, c.cols, ends_d[i].data_ptr(), len(c.ends), outs[i].data_ptr(),
+                c.cols, stream)
+        assert st == B.MX_OK, B.status_string(st)
+
+    s = torch.cuda.Stream()
+    for i in range(len(cases)):     # first calls set kernel attributes, outside capture
+        call(i, s.cuda_stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for i in range(len(cases)):
+                call(i, s.cuda_stream)
+    for rep in range(3):
+        if rep == 2:
+            # other group ends, the same blocked buffers read under them
+            c = cases[0]
+            new = synth.ends_from_sizes(synth.split_distinct_cuts(rng, c.cols, len(c.ends)))
+            ends_d[0].copy_(torch.from_numpy(new))
+            cases[0] = synth.Case(c.name, c.dim, c.scales, new, c.seed)
+        for o in outs:
+            o.fill_(0x5A)
+        g.replay()
+        torch.cuda.synchronize()
+        for i, c in enumerate(cases):
+            want = orc.inverse(c.dim, blocked[i].cpu().numpy(), c.rows, c.cols, c.ends)
+            assert np.array_equal(outs[i].cpu().numpy(), want), (rep, c.name)
+    del g
