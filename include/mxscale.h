@@ -59,7 +59,10 @@
  * Contexts.  The library uses the CUDA context current in the calling
  * thread.  Only when no context is current does it bind the current
  * device's primary context (as the CUDA runtime would); a context the caller
- * made current, primary or not, is left in place.
+ * made current, primary or not, is left in place.  Kernel attributes (the
+ * shared-memory sizes) are set once per device, in the context current at
+ * the library's first call on that device: make every call on a device from
+ * that same context (normally the primary one).
  */
 #ifndef MXSCALE_H
 #define MXSCALE_H
