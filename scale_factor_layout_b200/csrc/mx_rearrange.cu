@@ -254,7 +254,10 @@ rearrange_tma_k(const __grid_constant__ CUtensorMap tmap, const int32_t *__restr
         tma_load_2d(stages + st * kStageBytes, &tmap, it.x, it.y, &full[st]);
     };
 
-    // Thread 0 writes the staged tiles of an item, one bulk copy per group piece.
+    // Thread 0 writes the staged tiles of an item, one bulk copy per group
+    // piece, marking the lines first to evict from L2 (this kernel does not
+    // read its output; 1-2% over the default policy on a B200).
+    const uint64_t policy = policy_evict_first();
     auto store_item = [&](const KItem &it, const uint8_t *stg) {
         int g = it.g0;
         for (int t = 0; t < it.ntiles;) {
@@ -264,7 +267,7 @@ rearrange_tma_k(const __grid_constant__ CUtensorMap tmap, const int32_t *__restr
             const int W = table.pstart[g + 1] - table.pstart[g];
             const int64_t dst = (int64_t)s.padded_rows * table.pstart[g] + (int64_t)it.rb * kTileRows * W +
                                 (int64_t)(tau - (table.pstart[g] >> 2)) * 512;
-            bulk_store_s2g(out + dst, stg + t * 512, (uint32_t)(end - tau) * 512u);
+            bulk_store_s2g_hint(out + dst, stg + t * 512, (uint32_t)(end - tau) * 512u, policy);
             t = end - it.tau0;
             ++g;
         }
