@@ -800,7 +800,28 @@ unrearrange_box_k_kernel(const __grid_constant__ CUtensorMap omap, const uint8_t
             uint4 o[4];
 #pragma unroll
             for (int a = 0; a < 4; ++a) o[a] = make_uint4(0u, 0u, 0u, 0u);
-            if (it.np > 0 && cc0 < it.x + it.ncols) {
+            int kf = -1;   // the piece that holds all 16 columns of the chunk, if one does
+            for (int k = 0; k < it.np; ++k)
+                if (it.p[k].c0 <= cc0 && cc0 + 16 <= it.p[k].c1) kf = k;
+            if (kf >= 0) {
+                // the common case: no seam and no column past the box in the
+                // chunk, so every tile line read lies in the piece's loaded run
+                // (the fifth only when the chunk starts inside a tile)
+                const BoxPiece &p = it.p[kf];
+                const int u = cc0 - p.b;
+                const int sh = (u & 3) * 8;
+                const uint8_t *ln = stage + (p.s0 + (u >> 2) - p.f) * 512 + 16 * j;
+                uint4 w[5];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) w[t] = *reinterpret_cast<const uint4 *>(ln + t * 512);
+                w[4] = sh != 0 ? *reinterpret_cast<const uint4 *>(ln + 4 * 512) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    const uint32_t x0 = word_of(w[0], a), x1 = word_of(w[1], a), x2 = word_of(w[2], a),
+                                   x3 = word_of(w[3], a), x4 = word_of(w[4], a);
+                    o[a] = make_uint4(funnel(x0, x1, sh), funnel(x1, x2, sh), funnel(x2, x3, sh), funnel(x3, x4, sh));
+                }
+            } else if (it.np > 0 && cc0 < it.x + it.ncols) {
                 for (int k = 0; k < it.np; ++k) {
                     const BoxPiece &p = it.p[k];
                     if (p.c1 <= cc0 || p.c0 >= cc0 + 16) continue;
