@@ -108,6 +108,23 @@ def test_inverse_k_output_boxes(mxlib, orc, seed):
         _inverse_check(case, orc, out_pad=pad, misalign=0)
 
 
+@pytest.mark.parametrize("unit", [1, 4, 16, 128])
+def test_inverse_k_boxes_seam_alignment(mxlib, orc, unit):
+    """Output boxes whose group seams all fall on multiples of `unit` columns:
+    with 16 and 128 every 16-column output chunk lies inside one group and
+    starts on a tile boundary (the path with no shift and no seam merge); with
+    4 the seams sit on tiles but inside chunks; with 1 anywhere.  The last 48
+    columns belong to no group when the groups cover only whole units."""
+    rng = np.random.default_rng(4700 + unit)
+    rows, cols = 389, 1072
+    covered = cols - cols % unit if unit > 1 else cols
+    widths = synth.split_units(rng, covered, 8, unit)
+    scales = rng.integers(1, 255, size=(rows, cols), dtype=np.uint8)
+    case = synth.Case(f"seams{unit}K", synth.DIM_K, scales, np.cumsum(widths).astype(np.int32), 0)
+    for pad in (0, 16):
+        _inverse_check(case, orc, out_pad=pad, misalign=0)
+
+
 def test_inverse_ignores_padding_values(mxlib, orc):
     """Padding bytes of the blocked buffer (and its tail) filled with garbage
     change nothing: the inverse reads whole tiles but writes only real data."""
