@@ -595,41 +595,52 @@ def sweep_launches(traffic_bytes: int) -> int:
     return int(min(2000, max(20, SWEEP_GRAPH_SECONDS / est)))
 
 
-def oracle_seconds(case) -> tuple[float, str]:
-    """Single-thread CPU oracle time of one full call: the median of 3 runs
-    (each repeated to at least 20 ms for tiny points), or one run above
+def oracle_seconds(case, op: str = "rearrange") -> tuple[float, str]:
+    """Single-thread CPU oracle time of one full call (the rearrange, or the
+    inverse of the oracle's own blocked output): the median of 3 runs (each
+    repeated to at least 20 ms for tiny points), or one run above
     SWEEP_ORACLE_SINGLE_RUN bytes of traffic."""
     import oracle
 
     oracle.load()
+    if op == "inverse":
+        blocked = oracle.rearrange(case.dim, case.scales, case.ends)
+
+        def call():
+            oracle.inverse(case.dim, blocked, case.rows, case.cols, case.ends)
+    else:
+        def call():
+            oracle.rearrange(case.dim, case.scales, case.ends)
     b = algorithmic_bytes(case)
     if b["read"] + b["written"] > SWEEP_ORACLE_SINGLE_RUN:
         t0 = time.perf_counter()
-        oracle.rearrange(case.dim, case.scales, case.ends)
+        call()
         return time.perf_counter() - t0, "1 run"
     t0 = time.perf_counter()
-    oracle.rearrange(case.dim, case.scales, case.ends)
+    call()
     once = max(time.perf_counter() - t0, 1e-7)
     reps = max(1, int(math.ceil(0.02 / once)))
     runs = []
     for _ in range(3):
         t0 = time.perf_counter()
         for _ in range(reps):
-            oracle.rearrange(case.dim, case.scales, case.ends)
+            call()
         runs.append((time.perf_counter() - t0) / reps)
     return statistics.median(runs), f"median of 3 runs of {reps}"
 
 
 def run_sweep(args, rank, world, device, dist):
-    """Every point of the K-groups sweep, one after another: per point, its
-    launches back to back in one uploaded graph over a rotation of input and
-    output copies (one untimed replay, one timed), a same-size device copy
-    timed the same way, and the CPU oracle on the host."""
+    """Every point of the K-groups sweep, one after another (the rearrange, or
+    with --op inverse the inverse): per point, its launches back to back in
+    one uploaded graph over a rotation of input and output copies (one
+    untimed replay, one timed), a device copy of the same input timed the
+    same way, and the CPU oracle on the host."""
     import torch
 
     from scale_factor_layout_b200 import synth
 
     peak, peak_src = load_peaks()
+    op = args.op
     stream = torch.cuda.Stream(device)
     h = stream.cuda_stream
     timer = GraphTimer(stream, dist, device)
@@ -643,14 +654,15 @@ def run_sweep(args, rank, world, device, dist):
             traffic = b["read"] + b["written"]
             per_copy = b["read"] + b["alloc"]
             n_rot = min(max(2, math.ceil(4 * L2_BYTES / per_copy)), SWEEP_MAX_COPIES)
-            rot = device_copies(case, n_rot, device)
+            rot = device_copies(case, n_rot, device, op)
             with torch.cuda.stream(stream):
-                launch(rot[0], h)
+                launch(rot[0], h, op)
             n = sweep_launches(traffic)
-            g = timer.capture([lambda it=rot[k % n_rot]: launch(it, h) for k in range(n)])
+            g = timer.capture([lambda it=rot[k % n_rot]: launch(it, h, op) for k in range(n)])
             t = timer.steady(g, n)
             del g
             srcs = [it[1] for it in rot]
+            copy_bytes = 2 * srcs[0].numel()
             dsts = [torch.empty_like(x) for x in srcs]
             g = timer.capture([lambda a=srcs[k % n_rot], d=dsts[k % n_rot]: d.copy_(a) for k in range(n)])
             t_copy = timer.steady(g, n)
@@ -663,10 +675,10 @@ def run_sweep(args, rank, world, device, dist):
                      "gbps_pages_convention": round(per_copy / t / 1e9, 1),
                      "read_bytes": b["read"], "written_bytes": b["written"], "alloc_bytes": b["alloc"],
                      "copy_us": round(t_copy * 1e6, 3),
-                     "frac_of_copy": round((traffic / t) / (2 * case.rows * case.cols / t_copy), 4),
+                     "frac_of_copy": round((traffic / t) / (copy_bytes / t_copy), 4),
                      "launches_timed": n, "rotation": n_rot, "l2_cold": n_rot * per_copy >= 4 * L2_BYTES}
             if rank == 0 and not args.no_cpu_baseline:
-                ts, how = oracle_seconds(case)
+                ts, how = oracle_seconds(case, op)
                 entry.update({"oracle_us": round(ts * 1e6, 1), "oracle_gbps": round(traffic / ts / 1e9, 3),
                               "oracle_runs": how})
             points.append(entry)
@@ -680,7 +692,7 @@ def run_sweep(args, rank, world, device, dist):
         "steps": 1, "warmup": args.warmup, "ms_per_step": round(total_s * 1e3, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
         "data": "synthetic (seeded uniform E8M0 bytes, seeded group splits)",
-        "config": {"workload": "k_sweep", "op": "rearrange", "path": "auto",
+        "config": {"workload": "k_sweep", "op": op, "path": "auto",
                    "description": "K-groups sweep: M in {128..28672} x TotalK in {2^10..2^19}, scales M x TotalK/32, "
                                   "G=8 (70 points); a step is one pass over every point",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -693,8 +705,8 @@ def run_sweep(args, rank, world, device, dist):
         "frac_of_peak": round(total_bytes / total_s / 1e9 / peak, 4),
         "points": points,
         "large_points_min_frac_of_peak": min((p["frac_of_peak"] for p in big), default=None),
-        "roofline": roofline_entry("rearrange_tma_k", "k_sweep, all points", total_bytes, total_s, peak, peak_src,
-                                   None),
+        "roofline": roofline_entry("unrearrange_box_k_kernel" if op == "inverse" else "rearrange_tma_k",
+                                   "k_sweep, all points", total_bytes, total_s, peak, peak_src, None),
         "e2e": None,
         "gpu_launches": launches,
         "clocks": sampler.summary(),

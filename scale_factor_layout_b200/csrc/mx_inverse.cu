@@ -591,8 +591,8 @@ unrearrange_tma_m_kernel(const __grid_constant__ CUtensorMap omap, int64_t map_w
 // shift give the bytes, as in the shift-mode transpose above; a chunk that
 // holds a seam merges the pieces' bytes by column.  Columns no group covers
 // are zero.  A box with more pieces than kBoxPieces, or more tiles than a
-// stage holds (groups narrower than about 40 columns), is gathered byte by
-// byte from global memory instead.  Items go in group-major order (the boxes
+// stage holds (groups narrower than about 40 columns), reads the same tile
+// lines straight from global memory instead, group by group.  Items go in group-major order (the boxes
 // whose first column lies in group 0, band after band, then group 1's, ...),
 // so that the items in flight read one stretch of the blocked buffer, which
 // lets each CTA prefetch its likely first tiles into L2 before its group
@@ -615,7 +615,7 @@ struct BoxPiece {
 struct BoxItem {
     int32_t x, y;     // first output column (a multiple of 128) and row
     int32_t ncols;    // columns of the box inside the output (<= 128)
-    int32_t np;       // pieces, or -1: gather the box from global memory
+    int32_t np;       // pieces, or -1: read the box's tile lines from global memory
     int32_t rb;       // row band
     int32_t tiles;    // tiles loaded into the stage
     BoxPiece p[kBoxPieces];
@@ -857,24 +857,45 @@ unrearrange_box_k_kernel(const __grid_constant__ CUtensorMap omap, const uint8_t
                     }
                 }
             } else if (it.np < 0 && cc0 < it.x + it.ncols) {
-                // many narrow groups: each byte straight from the blocked buffer
-                const int lim = min(table.begin[s.G - 1] + table.size[s.G - 1], it.x + it.ncols);
+                // More, narrower groups than a stage holds: per group that meets
+                // the chunk, the same tile lines, shift and column masks as
+                // above, read straight from the blocked buffer (a warp reads
+                // whole 512-byte tiles).
+                const int cend = min(cc0 + 16, it.x + it.ncols);
+                for (int g = find_group_col(table, s.G, cc0); g < s.G && table.begin[g] < cend; ++g) {
+                    const int b = table.begin[g], wg = table.size[g];
+                    if (wg == 0 || b + wg <= cc0) continue;
+                    const int u = cc0 - b;              // local column of the chunk's byte 0 (may be < 0)
+                    const int t0 = u >> 2;              // floor
+                    const int sh = (u & 3) * 8;
+                    const int ntg = (wg + 3) >> 2;      // the group's tiles in a row band
+                    const uint8_t *lines = blocked + box_src(table, s, g, it.rb, 0) + 16 * j;
+                    uint4 w[5];
 #pragma unroll
-                for (int a = 0; a < 4; ++a) {
-                    const int r = j + 32 * a;
-                    uint32_t wv[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const int c = cc0 + k;
-                        if (c < lim) {
-                            const int g = find_group_col(table, s.G, c);
-                            const int l = c - table.begin[g];
-                            const uint8_t v = __ldg(blocked + box_src(table, s, g, it.rb, l >> 2) + (r & 31) * 16 +
-                                                    (r >> 5) * 4 + (l & 3));
-                            wv[k >> 2] |= (uint32_t)v << (8 * (k & 3));
-                        }
+                    for (int t = 0; t < 5; ++t) {
+                        const int tl = t0 + t;
+                        w[t] = (tl >= 0 && tl < ntg && (t < 4 || sh != 0))
+                                   ? __ldg(reinterpret_cast<const uint4 *>(lines + 512 * tl))
+                                   : make_uint4(0u, 0u, 0u, 0u);
                     }
-                    o[a] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                    const int k0 = max(b - cc0, 0), k1 = min(b + wg, cend) - cc0;
+                    uint32_t keep[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int lo = min(max(k0 - 4 * e, 0), 4), hi = min(max(k1 - 4 * e, 0), 4);
+                        const uint32_t upto_hi = hi == 4 ? 0xffffffffu : (1u << (8 * hi)) - 1u;
+                        const uint32_t below_lo = lo == 4 ? 0xffffffffu : (1u << (8 * lo)) - 1u;
+                        keep[e] = upto_hi & ~below_lo;
+                    }
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        const uint32_t x0 = word_of(w[0], a), x1 = word_of(w[1], a), x2 = word_of(w[2], a),
+                                       x3 = word_of(w[3], a), x4 = word_of(w[4], a);
+                        o[a].x |= funnel(x0, x1, sh) & keep[0];
+                        o[a].y |= funnel(x1, x2, sh) & keep[1];
+                        o[a].z |= funnel(x2, x3, sh) & keep[2];
+                        o[a].w |= funnel(x3, x4, sh) & keep[3];
+                    }
                 }
             }
 #pragma unroll
