@@ -109,3 +109,14 @@ def test_timing_graph_sizes():
     assert bench.sweep_launches(8192) == 2000
     assert bench.sweep_launches(940_000_000) == 84
     assert bench.sweep_launches(10**12) == 20
+
+
+def test_oracle_seconds_times_either_op():
+    """The sweep's CPU leg times the oracle's rearrange, or its inverse of the
+    oracle's own blocked output, on the host (no GPU)."""
+    from scale_factor_layout_b200 import synth
+
+    case = synth.k_sweep_point(0, 0)   # 128 x 32 scale columns, G=8
+    for op in ("rearrange", "inverse"):
+        t, how = bench.oracle_seconds(case, op)
+        assert t > 0 and how.startswith("median of 3 runs of ")
