@@ -383,12 +383,22 @@ rearrange_tma_k(const __grid_constant__ CUtensorMap tmap, const int32_t *__restr
 // 16-byte boundary at or below its first byte (boxes past the array's end
 // read zeros).  Rows sit at pitch row_stride in shared memory; with the
 // stride a multiple of 4 every row starts on a word, and the transpose reads
-// 32-bit words.  Pipeline, staging and bulk stores follow rearrange_tma_m.
+// 32-bit words.  The pipeline follows rearrange_tma_m.  An item's output is
+// one contiguous span of whole tiles, so a warp can write its tiles' lines
+// straight from registers with 16-byte stores that cover whole 512-byte
+// tiles (kDirect), or stage them for one bulk copy per item as
+// rearrange_tma_m does.
 //
-// Two instances: 8 warps and 4 stages for rows of more than 64 padded
-// columns; 4 warps and 2 stages for rows of at most 64 (one quad of tiles
-// per warp), small enough per CTA that about one row block per CTA is
-// resident at once on a B200 (1032 row blocks of a 131072-row input).
+// Instances: 8 warps, 4 stages and direct stores for rows of more than 64
+// padded columns (no staging blocks, so twice the CTAs per SM: 27-32%
+// faster than staged bulk stores from 131072 to 1048576 rows of 100-200
+// columns on a B200); 4 warps and 2 stages for rows of at most 64 (one quad
+// of tiles per warp), small enough per CTA that about one row block per CTA
+// is resident at once (1032 row blocks of a 131072-row input).  The 4-warp
+// kernel stores directly when the items fit in two waves of the grid (the
+// store leaves the critical path of a CTA's one or two items: 5-8% faster
+// up to 262144 rows of 44 columns) and stages bulk copies otherwise (3-5%
+// faster from 524288 rows, where each CTA streams several items).
 constexpr int kFlatBoxWords = 256;
 constexpr int kFlatBoxBytes = kFlatBoxWords * 4;
 constexpr int kFlatStages = 4;
@@ -398,10 +408,10 @@ constexpr int kFlatNarrowCols = 64;   // padded columns up to which the 4-warp i
 struct FlatShape {
     int32_t row_stride;     // bytes, a multiple of 4
     int32_t stage_bytes;    // boxes per stage * 1 KB
-    int32_t staging_bytes;  // tiles per row block * 512, rounded to 1 KB
+    int32_t staging_bytes;  // tiles per row block * 512, rounded to 1 KB (staged instances only)
 };
 
-template <int kWarpsF, int kStagesF>
+template <int kWarpsF, int kStagesF, bool kDirect>
 __global__ void __launch_bounds__(kWarpsF * 32)
 rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__restrict__ ends,
                    uint8_t *__restrict__ out, int64_t out_size, Shape s, FlatShape f) {
@@ -501,7 +511,7 @@ rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__re
                 }
             }
         }
-        if (tid == 0) bulk_wait_read<0>();
+        if (!kDirect && tid == 0) bulk_wait_read<0>();
         if (__syncthreads_or(!ok)) {
             if (tid == 0) {
                 atomicOr(&g_mx_flags, kFlagWaitTimeout);
@@ -512,14 +522,17 @@ rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__re
         }
         if (tid == 0) {
             if (refill) issue(next, st);
-            if (n > 0) {
-                bulk_store_s2g(out + prev_off, staging + ((n - 1) & 1) * f.staging_bytes, prev_bytes);
-                bulk_commit();
+            if (!kDirect) {
+                if (n > 0) {
+                    bulk_store_s2g(out + prev_off, staging + ((n - 1) & 1) * f.staging_bytes, prev_bytes);
+                    bulk_commit();
+                }
+                prev_off = it.out_off;
+                prev_bytes = (uint32_t)it.ntiles * 512u;
             }
-            prev_off = it.out_off;
-            prev_bytes = (uint32_t)it.ntiles * 512u;
         }
-        uint8_t *stg = staging + (n & 1) * f.staging_bytes;
+        // the item's tiles: straight to the output, or into staging block n % 2
+        uint8_t *stg = kDirect ? out + it.out_off : staging + (n & 1) * f.staging_bytes;
 #pragma unroll
         for (int p = 0; p < kPasses; ++p) {
             const int qq = q + kWarpsF * p;
@@ -537,9 +550,9 @@ rearrange_flat_tma(const __grid_constant__ CUtensorMap tmap, const int32_t *__re
                 }
             }
         }
-        fence_proxy_async_smem();
+        if (!kDirect) fence_proxy_async_smem();
     }
-    if (n_my > 0) {
+    if (!kDirect && n_my > 0) {
         __syncthreads();
         if (tid == 0) {
             bulk_store_s2g(out + prev_off, staging + ((n_my - 1) & 1) * f.staging_bytes, prev_bytes);
@@ -662,7 +675,9 @@ FlatShape flat_shape(int64_t row_stride, int64_t padded_cols) {
     return f;
 }
 
-int flat_smem_bytes(const FlatShape &f, int stages) { return stages * f.stage_bytes + 2 * f.staging_bytes + 128; }
+int flat_smem_bytes(const FlatShape &f, int stages, bool direct) {
+    return stages * f.stage_bytes + (direct ? 0 : 2 * f.staging_bytes) + 128;
+}
 
 // The flat kernel instance for rows of `padded_cols` columns.
 bool flat_narrow(int64_t padded_cols) { return padded_cols <= kFlatNarrowCols; }
@@ -726,13 +741,15 @@ mx_status device_info(const DeviceInfo **out) {
     if (!d.ready) {
         if (cudaError_t e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev); e != cudaSuccess)
             return cuda_status(e);
-        const int flat_max = flat_smem_bytes(flat_shape(kFlatMaxStride, kFlatMaxStride), kFlatStages);
-        const int flat_narrow_max = flat_smem_bytes(flat_shape(kFlatMaxStride, kFlatNarrowCols), 2);
+        const int flat_max = flat_smem_bytes(flat_shape(kFlatMaxStride, kFlatMaxStride), kFlatStages, true);
+        const FlatShape narrow_max = flat_shape(kFlatMaxStride, kFlatNarrowCols);
         const cudaError_t setup[] = {
-            cudaFuncSetAttribute(rearrange_flat_tma<8, kFlatStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(rearrange_flat_tma<8, kFlatStages, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  flat_max),
-            cudaFuncSetAttribute(rearrange_flat_tma<4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 flat_narrow_max),
+            cudaFuncSetAttribute(rearrange_flat_tma<4, 2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 flat_smem_bytes(narrow_max, 2, true)),
+            cudaFuncSetAttribute(rearrange_flat_tma<4, 2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 flat_smem_bytes(narrow_max, 2, false)),
             cudaFuncSetAttribute(rearrange_tma_m, cudaFuncAttributeMaxDynamicSharedMemorySize, tma_smem_bytes<true>()),
             cudaFuncSetAttribute(rearrange_tma_k, cudaFuncAttributeMaxDynamicSharedMemorySize, tma_smem_bytes<false>()),
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_tma[1], rearrange_tma_m, kThreads,
@@ -876,13 +893,24 @@ mx_status run(mx_group_dim dim, const uint8_t *scales, int64_t rows, int64_t col
         if (r != CUDA_SUCCESS) return cuda_status(static_cast<cudaError_t>(r));   // driver code
         const FlatShape f = flat_shape(row_stride, s.padded_cols);
         const bool narrow = flat_narrow(s.padded_cols);
-        auto kernel = narrow ? rearrange_flat_tma<4, 2> : rearrange_flat_tma<8, kFlatStages>;
         const int block = narrow ? 128 : kThreads;
-        const int smem = flat_smem_bytes(f, narrow ? 2 : kFlatStages);
+        const int stages = narrow ? 2 : kFlatStages;
+        // Direct stores, except for the 4-warp kernel when the items outnumber
+        // two waves of the grid (each CTA then streams several items, and the
+        // staged bulk stores overlap them better).
+        auto kernel = narrow ? rearrange_flat_tma<4, 2, true> : rearrange_flat_tma<8, kFlatStages, true>;
+        int smem = flat_smem_bytes(f, stages, true);
         int occ = 0;
         if (cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, block, smem);
             e != cudaSuccess || occ < 1)
             return cuda_status(e != cudaSuccess ? e : cudaErrorInvalidConfiguration);
+        if (narrow && work > 2ll * d->sms * occ) {
+            kernel = rearrange_flat_tma<4, 2, false>;
+            smem = flat_smem_bytes(f, stages, false);
+            if (cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, block, smem);
+                e != cudaSuccess || occ < 1)
+                return cuda_status(e != cudaSuccess ? e : cudaErrorInvalidConfiguration);
+        }
         const int64_t cap = (int64_t)d->sms * occ;
         const int grid = (int)(work < cap ? work : cap);
         launched = launch_kernel_block(kernel, grid, block, smem, stream, map, ends, out, (int64_t)size, s, f);

@@ -53,6 +53,22 @@ def test_workloads_forced_path(mxlib, orc, cases, name, path):
     _check(cases[name], orc, path)
 
 
+@pytest.mark.parametrize("rows,cols", [(262144, 44), (600000, 44), (700000, 60), (40000, 100), (40000, 252)])
+def test_flat_instances(mxlib, orc, rows, cols):
+    """The flat-row kernel's instances at the sizes where each is chosen:
+    4 warps with direct stores (up to two waves of items: 262144 rows) and
+    with staged bulk stores (more: 600000 and 700000 rows), and 8 warps with
+    direct stores for rows of 65-256 padded columns; the row stride is the
+    column count (a multiple of 4, not of 16)."""
+    rng = np.random.default_rng(5100 + cols + rows)
+    scales = rng.integers(1, 255, size=(rows, cols), dtype=np.uint8)
+    sizes = synth.split_multinomial(rng, rows, 8)
+    case = synth.Case(f"flat{rows}x{cols}", synth.DIM_M, scales, np.cumsum(sizes).astype(np.int32), 0)
+    dc = DeviceCase(case)
+    assert B.mx_select_path(case.dim, dc.ptr, case.rows, case.cols, case.row_stride) == B.MX_PATH_FLAT
+    _check(case, orc, "auto")
+
+
 def test_auto_dispatch_choices(mxlib, cases):
     for name, want in (("m_tiny", B.MX_PATH_FLAT), ("m_skinny", B.MX_PATH_FLAT),
                        ("m_wide", B.MX_PATH_TMA), ("k_groups", B.MX_PATH_TMA)):
