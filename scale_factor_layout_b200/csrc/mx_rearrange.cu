@@ -389,10 +389,11 @@ rearrange_tma_k(const __grid_constant__ CUtensorMap tmap, const int32_t *__restr
 // tiles (kDirect), or stage them for one bulk copy per item as
 // rearrange_tma_m does.
 //
-// Instances: 8 warps, 4 stages and direct stores for rows of more than 64
-// padded columns (no staging blocks, so twice the CTAs per SM: 27-32%
-// faster than staged bulk stores from 131072 to 1048576 rows of 100-200
-// columns on a B200); 4 warps and 2 stages for rows of at most 64 (one quad
+// Instances: 8 warps, 2 stages and direct stores for rows of more than 64
+// padded columns (no staging blocks and two stages, so up to four times the
+// CTAs per SM of four stages with staging: 131072x100 7.2 vs 9.8 us,
+// 131072x200 10.3 vs 18.1, 1048576x200 72 vs 108 on a B200); 4 warps and 2
+// stages for rows of at most 64 (one quad
 // of tiles per warp), small enough per CTA that about one row block per CTA
 // is resident at once (1032 row blocks of a 131072-row input).  The 4-warp
 // kernel stores directly when the items fit in two waves of the grid (the
@@ -401,7 +402,7 @@ rearrange_tma_k(const __grid_constant__ CUtensorMap tmap, const int32_t *__restr
 // faster from 524288 rows, where each CTA streams several items).
 constexpr int kFlatBoxWords = 256;
 constexpr int kFlatBoxBytes = kFlatBoxWords * 4;
-constexpr int kFlatStages = 4;
+constexpr int kFlatStages = 2;
 constexpr int kFlatMaxStride = 256;
 constexpr int kFlatNarrowCols = 64;   // padded columns up to which the 4-warp instance runs
 
